@@ -1,0 +1,385 @@
+"""Pins of the CPU oracle to facts outside itself (pages' printed values,
+closed forms, invariants, library routines). CPU only."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import klein_inputs as ki
+import oracle as o
+
+
+# ---------------------------------------------------------------- schedule
+
+def test_schedule_16_printed_values(golden):
+    g = golden("schedule_16.txt")
+    s = o.sigma_schedule(16)
+    assert len(s) == 17 and s[-1] == 0.0
+    np.testing.assert_allclose(np.round(s[:3], 3), g["first"], atol=0)
+    np.testing.assert_allclose(np.round(s[13:16], 3), g["last"], atol=0)
+    assert round(s[0] - s[1], 3) == g["first_step"]
+    assert round(s[15] - s[16], 3) == g["last_step"]
+    assert int((s[:-1] > 0.5).sum()) == g["above_half"]
+
+
+def test_schedule_other_printed_values(golden):
+    g = golden("schedule_other.txt")
+    s50 = o.sigma_schedule(50, g["shift"])
+    assert int((s50[:-1] > 0.5).sum()) == g["steps50_above_half"]
+    # "step 10": both 0-based and 1-based readings round to 0.97
+    assert round(s50[9], 2) == g["steps50_step10"]
+    assert round(s50[10], 2) == g["steps50_step10"]
+    s4 = o.sigma_schedule(4)
+    assert round(s4[3], 3) == g["steps4_last"] and s4[4] == 0.0
+
+
+def test_schedule_shift_one_is_linear():
+    # shift 1 leaves the evenly spaced levels unchanged (closed form)
+    np.testing.assert_allclose(o.sigma_schedule(8, 1.0)[:-1], np.linspace(1, 1 / 8, 8), rtol=0, atol=1e-15)
+
+
+def test_timesteps_scale():
+    np.testing.assert_allclose(o.timesteps([1.0, 0.5, 0.0]), [1000.0, 500.0, 0.0])
+
+
+# ------------------------------------------------------------- geometry
+
+def test_token_counts(golden):
+    g = golden("structure.txt")
+    assert o.image_tokens(1024, 1024) == g["tokens_1024x1024"]
+    assert o.image_tokens(4096, 4096) == g["tokens_4096x4096"]
+    assert o.image_tokens(1024, 1024) == g["ref_tokens_1024x1024"]
+    assert o.image_tokens(128, 128) == 64
+    assert o.image_tokens(2048, 2048) == 16384
+    assert 512 + 2 * o.image_tokens(1024, 1024) == 8704
+
+
+def test_text_padding(golden):
+    g = golden("structure.txt")
+    assert o.TEXT_PAD == g["text_pad"]
+    assert [o.pad_text_len(n) for n in (1, 79, 80, 81, 160, 512)] == [80, 80, 80, 160, 160, 560]
+    assert 8 * 2560 == g["text_stack_dim"]
+
+
+def test_positions_table():
+    p = o.positions(3, (2, 2), refs=((1, 2), (1, 1)))
+    expect = [(0, 0, 0, 0), (0, 0, 0, 1), (0, 0, 0, 2),
+              (0, 0, 0, 0), (0, 0, 1, 0), (0, 1, 0, 0), (0, 1, 1, 0),
+              (0, 0, 0, -1), (0, 0, 1, -1), (0, 0, 0, -2)]
+    np.testing.assert_array_equal(p, np.array(expect, float))
+
+
+def test_parameter_counts(golden):
+    g = golden("structure.txt")
+    assert o.parameter_count(False) == g["base_params"]
+    assert o.parameter_count(True) == g["distilled_params"]
+    assert o.parameter_count(True) - o.parameter_count(False) == g["param_diff"]
+    assert (o.DIM, o.HEADS, o.HEAD_DIM) == (g["dim"], g["heads"], g["head_dim"])
+    assert (o.N_STAGE1, o.N_JOINT, o.AXIS_DIM) == (g["stage1_blocks"], g["joint_blocks"], g["rope_axis_dims"])
+
+
+def test_generated_weights_match_parameter_layout():
+    # The generator's tensors, counted, equal the oracle's structural count
+    # (which is pinned to the printed totals) for a 1+1-block stack.
+    m = ki.ModelWeights(seed=0, distilled=True, n_stage1=1, n_joint=1)
+    n = sum(a.size for a in m.misc.values())
+    for mode in ki.MODES:
+        n += sum(a.size for a in m.stage1(mode)[0].values())
+    n += sum(a.size for a in m.joint()[0].values())
+    assert n == o.parameter_count(True, 1, 1, txt_in=False)
+
+
+# ------------------------------------------------------- embeddings
+
+def test_sinusoid_zero_and_period():
+    e = o.timestep_sinusoid(0.0)
+    np.testing.assert_array_equal(e[:128], 1.0)
+    np.testing.assert_array_equal(e[128:], 0.0)
+    # frequency 0 is 1 rad per unit of t: cos/sin of t itself
+    e = o.timestep_sinusoid(0.5)
+    assert e[0] == pytest.approx(math.cos(0.5)) and e[128] == pytest.approx(math.sin(0.5))
+    np.testing.assert_allclose(e[:128] ** 2 + e[128:] ** 2, 1.0, atol=1e-14)
+
+
+def test_silu_closed_form():
+    assert o.silu(0.0) == 0.0
+    assert o.silu(1.0) == pytest.approx(1 / (1 + math.exp(-1)))
+    assert o.silu(-50.0) == pytest.approx(0.0, abs=1e-18)
+
+
+def test_context_modes_ignore_image_time():
+    m = ki.ModelWeights(seed=0, distilled=False, n_stage1=1, n_joint=1)
+    a = o.stage_modulations(m.misc, 0.9, None)
+    b = o.stage_modulations(m.misc, 0.2, None)
+    for st in (1, 2):
+        np.testing.assert_array_equal(a[st][o.MODE_TXT], b[st][o.MODE_TXT])
+        np.testing.assert_array_equal(a[st][o.MODE_REF], b[st][o.MODE_REF])
+        assert not np.allclose(a[st][o.MODE_IMG], b[st][o.MODE_IMG])
+    # image at sigma 0 has the same embedding as the context streams
+    c = o.stage_modulations(m.misc, 0.0, None)
+    np.testing.assert_array_equal(c[1][o.MODE_IMG], o.modulation(m.misc["mod1.img"], o.time_embedding(m.misc, 0.0, None), 3))
+
+
+def test_target_embedder_adds_to_every_mode():
+    m = ki.ModelWeights(seed=0, distilled=True, n_stage1=1, n_joint=1)
+    e1 = o.time_embedding(m.misc, 0.5, 0.3)
+    e0 = o.time_embedding(m.misc, 0.5, None)
+    e_t = o.time_embed_mlp(m.misc["tt_mlp1"], m.misc["tt_mlp2"], 0.3)
+    np.testing.assert_allclose(e1, e0 + e_t, rtol=0, atol=1e-12)
+    # context streams at t=0 still see the target embedding
+    ctx = o.time_embedding(m.misc, 0.0, 0.3)
+    assert not np.allclose(ctx, o.time_embedding(m.misc, 0.0, None))
+
+
+# ------------------------------------------------------------ norms
+
+def test_layer_norm_moments():
+    x = np.random.default_rng(3).normal(2.0, 5.0, size=(7, o.DIM))
+    y = o.layer_norm(x)
+    np.testing.assert_allclose(y.mean(-1), 0.0, atol=1e-12)
+    np.testing.assert_allclose(y.var(-1), 1.0, rtol=1e-6)
+    # shift/scale invariance of a no-affine LayerNorm
+    np.testing.assert_allclose(o.layer_norm(3 * x + 7), y, atol=1e-9)
+
+
+def test_modln_modes():
+    rng = np.random.default_rng(4)
+    x = rng.normal(size=(1, 5, o.DIM))
+    mod = rng.normal(size=(3, 3, o.DIM))
+    modes = np.array([0, 0, 1, 2, 2])
+    h = o.modln(x, modes, mod)
+    xh = o.layer_norm(x)
+    for r, m in enumerate(modes):
+        np.testing.assert_allclose(h[0, r], (1 + mod[m, 1]) * xh[0, r] + mod[m, 0], atol=1e-12)
+    # scale = -1 makes every row equal to its mode's shift
+    mod2 = mod.copy()
+    mod2[:, 1] = -1.0
+    np.testing.assert_allclose(o.modln(x, modes, mod2)[0], mod2[modes, 0], atol=1e-12)
+
+
+def test_rms_norm_unit_rms():
+    x = np.random.default_rng(5).normal(0, 3, size=(4, 24, 128))
+    y = o.rms_norm(x, np.ones(128))
+    np.testing.assert_allclose(np.sqrt((y * y).mean(-1)), 1.0, rtol=1e-6)
+    w = np.random.default_rng(6).normal(size=128)
+    np.testing.assert_allclose(o.rms_norm(x, w), y * w, atol=1e-12)
+
+
+# ------------------------------------------------------------- RoPE
+
+def test_rope_preserves_pair_norms():
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=(9, 3, 128))
+    pos = rng.integers(-20, 600, size=(9, 4)).astype(float)
+    y = o.rope(x, pos)
+    nx = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    ny = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    np.testing.assert_allclose(ny, nx, rtol=1e-12)
+
+
+def test_rope_zero_position_is_identity():
+    x = np.random.default_rng(8).normal(size=(5, 2, 128))
+    np.testing.assert_array_equal(o.rope(x, np.zeros((5, 4))), x)
+
+
+def test_rope_relative_property():
+    rng = np.random.default_rng(9)
+    q = rng.normal(size=(1, 1, 128))
+    k = rng.normal(size=(1, 1, 128))
+    p1 = np.array([[0.0, 3.0, 5.0, 7.0]])
+    p2 = np.array([[0.0, 1.0, -2.0, 4.0]])
+    d = p1 - p2
+    a = np.sum(o.rope(q, p1) * o.rope(k, p2))
+    b = np.sum(o.rope(q, d) * o.rope(k, np.zeros((1, 4))))
+    assert a == pytest.approx(b, rel=1e-12)
+
+
+def test_rope_axis_blocks_and_frequencies():
+    # a position on one axis only rotates that axis' 32 dims; pair j of an
+    # axis turns by p * 10000^(-2j/32)
+    x = np.zeros((1, 1, 128))
+    x[..., 0::2] = 1.0
+    for axis in range(4):
+        pos = np.zeros((1, 4))
+        pos[0, axis] = 3.0
+        y = o.rope(x, pos)[0, 0]
+        for d in range(0, 128, 2):
+            a, j = divmod(d // 2, 16)
+            ang = 3.0 * 10000.0 ** (-2 * j / 32) if a == axis else 0.0
+            assert y[d] == pytest.approx(math.cos(ang), abs=1e-14)
+            assert y[d + 1] == pytest.approx(math.sin(ang), abs=1e-14)
+
+
+# -------------------------------------------------------- attention
+
+def test_attention_matches_library():
+    rng = np.random.default_rng(10)
+    q = rng.normal(size=(2, 13, 3, 128))
+    k = rng.normal(size=(2, 17, 3, 128))
+    v = rng.normal(size=(2, 17, 3, 128))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).transpose(1, 2), torch.from_numpy(k).transpose(1, 2),
+        torch.from_numpy(v).transpose(1, 2)).transpose(1, 2).numpy()
+    np.testing.assert_allclose(o.attention(q, k, v), ref, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(11)
+    k = rng.normal(size=(1, 6, 2, 128))
+    v = rng.normal(size=(1, 6, 2, 128))
+    # zero queries attend uniformly
+    out = o.attention(np.zeros((1, 4, 2, 128)), k, v)
+    np.testing.assert_allclose(out, np.broadcast_to(v.mean(1, keepdims=True), out.shape), atol=1e-14)
+    # a single key returns its value
+    out = o.attention(rng.normal(size=(1, 3, 2, 128)), k[:, :1], v[:, :1])
+    np.testing.assert_allclose(out, np.broadcast_to(v[:, :1], out.shape), atol=1e-14)
+
+
+def _brute_attention(q, k, v):
+    # scalar loops on a tiny case
+    Rq, Rk, d = q.shape[0], k.shape[0], q.shape[1]
+    out = np.zeros((Rq, d))
+    for i in range(Rq):
+        s = [sum(q[i, c] * k[j, c] for c in range(d)) / math.sqrt(d) for j in range(Rk)]
+        m = max(s)
+        e = [math.exp(t - m) for t in s]
+        z = sum(e)
+        for j in range(Rk):
+            out[i] += e[j] / z * v[j]
+    return out
+
+
+def test_attention_brute_force_tiny():
+    rng = np.random.default_rng(12)
+    q = rng.normal(size=(1, 4, 1, 128))
+    k = rng.normal(size=(1, 5, 1, 128))
+    v = rng.normal(size=(1, 5, 1, 128))
+    np.testing.assert_allclose(o.attention(q, k, v)[0, :, 0], _brute_attention(q[0, :, 0], k[0, :, 0], v[0, :, 0]), atol=1e-12)
+
+
+# ------------------------------------------------------------- block
+
+@pytest.fixture(scope="module")
+def small_block():
+    w = ki.block_weights(0, "pin.block")
+    n_txt, gh, gw = 6, 3, 4
+    pos = o.positions(n_txt, (gh, gw))
+    modes = o.mode_of_rows(n_txt, gh * gw, 0)
+    x = ki.tokens(1, "pin", 1, len(modes)).astype(np.float64)
+    mod = ki.modulation_vectors(1, "pin").astype(np.float64)
+    return w, pos, modes, x, mod
+
+
+def test_block_gate_zero_is_identity(small_block):
+    w, pos, modes, x, mod = small_block
+    m = mod.copy()
+    m[:, 2] = 0.0
+    np.testing.assert_array_equal(o.block(x, pos, modes, m, w), x)
+
+
+def test_block_linear_in_gate(small_block):
+    w, pos, modes, x, mod = small_block
+    m2 = mod.copy()
+    m2[:, 2] *= 2.0
+    d1 = o.block(x, pos, modes, mod, w) - x
+    d2 = o.block(x, pos, modes, m2, w) - x
+    np.testing.assert_allclose(d2, 2 * d1, rtol=1e-9, atol=1e-9)
+
+
+def test_block_constant_input_closed_form(small_block):
+    # scale = -1: every row of h equals its mode's shift. Give all modes the
+    # same shift c: all values are equal, so attention returns that value
+    # whatever the scores, and the block delta is gate * (W_o (W_v c) + W_d swiglu).
+    w, pos, modes, x, mod = small_block
+    c = np.random.default_rng(13).normal(size=o.DIM)
+    m = mod.copy()
+    m[:, 1] = -1.0
+    m[:, 0] = c
+    D, F = o.DIM, o.MLP_HIDDEN
+    w_in = w["w_in"].astype(np.float64)
+    w_out = w["w_out"].astype(np.float64)
+    v = w_in[2 * D:3 * D] @ c
+    g = w_in[3 * D:3 * D + F] @ c
+    u = w_in[3 * D + F:] @ c
+    delta = w_out[:, :D] @ v + w_out[:, D:] @ (g / (1 + np.exp(-g)) * u)
+    out = o.block(x, pos, modes, m, w)
+    np.testing.assert_allclose(out - x, m[modes, 2][None] * delta[None, None], rtol=1e-9, atol=1e-9)
+
+
+def test_block_zero_queries_attend_uniformly(small_block):
+    # With the q projection zeroed, q = 0 after RMSNorm and RoPE; the
+    # attention branch is then the mean value row through the out-projection.
+    w, pos, modes, x, mod = small_block
+    D = o.DIM
+    wz = dict(w)
+    wz["w_in"] = w["w_in"].copy()
+    wz["w_in"][0:D] = 0.0
+    wm = dict(wz)
+    wm["w_out"] = w["w_out"].copy()
+    wm["w_out"][:, D:] = 0.0          # attention branch only
+    h = o.modln(x, modes, mod)
+    vbar = (h[0] @ w["w_in"][2 * D:3 * D].astype(np.float64).T).mean(0)
+    expect = mod[modes, 2] * (w["w_out"][:, :D].astype(np.float64) @ vbar)[None]
+    np.testing.assert_allclose(o.block(x, pos, modes, mod, wm)[0] - x[0], expect, rtol=1e-9, atol=1e-9)
+
+
+def test_block_permutation_equivariance(small_block):
+    w, pos, modes, x, mod = small_block
+    perm = np.random.default_rng(14).permutation(len(modes))
+    a = o.block(x, pos, modes, mod, w)[:, perm]
+    b = o.block(x[:, perm], pos[perm], modes[perm], mod, w)
+    np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+
+
+def test_block_row_subset(small_block):
+    w, pos, modes, x, mod = small_block
+    rows = np.array([0, 5, 7, 17])
+    np.testing.assert_allclose(o.block(x, pos, modes, mod, w, rows=rows),
+                               o.block(x, pos, modes, mod, w)[:, rows], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------ sampler pieces
+
+def test_euler_constant_velocity_lands_on_x0():
+    rng = np.random.default_rng(15)
+    x0 = rng.normal(size=(10, 128))
+    eps = rng.normal(size=(10, 128))
+    for steps in (1, 4, 16, 50):
+        s = o.sigma_schedule(steps)
+        x = eps.copy()
+        for i in range(steps):
+            x = o.euler_step(x, eps - x0, s[i], s[i + 1])
+        np.testing.assert_allclose(x, x0, atol=1e-12)
+        # x0 preview at sigma = 1 recovers x0 exactly from the true velocity
+        np.testing.assert_allclose(o.x0_preview(eps, eps - x0, 1.0), x0, atol=1e-12)
+
+
+def test_euler_zero_velocity():
+    x = np.random.default_rng(16).normal(size=(3, 128))
+    np.testing.assert_array_equal(o.euler_step(x, np.zeros_like(x), 0.7, 0.3), x)
+
+
+def test_cfg_limits():
+    rng = np.random.default_rng(17)
+    vc, vu = rng.normal(size=(2, 5, 128))
+    np.testing.assert_allclose(o.cfg_combine(vc, vu, 1.0), vc, rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(o.cfg_combine(vc, vu, 0.0), vu)
+    np.testing.assert_allclose(o.cfg_combine(vc, vu, 3.5), vu + 3.5 * (vc - vu))
+
+
+# ------------------------------------------------------------- stack
+
+def test_stage1_streams_are_isolated():
+    m = ki.ModelWeights(seed=0, distilled=False, n_stage1=1, n_joint=1)
+    n_txt, gh, gw = 5, 2, 3
+    pos = o.positions(n_txt, (gh, gw))
+    text = ki.text_embeddings(1, 1, n_txt)
+    lat_a = ki.noise_latents(2, gh * gw)
+    lat_b = ki.noise_latents(3, gh * gw)
+    sa, sb = {}, {}
+    o.transformer(m, lat_a, text, None, pos, 0.8, None, stage1_out=sa)
+    o.transformer(m, lat_b, text, None, pos, 0.3, None, stage1_out=sb)
+    # text stage-1 output ignores the image's latents and noise level
+    np.testing.assert_array_equal(sa["txt"], sb["txt"])
+    assert not np.allclose(sa["img"], sb["img"])
