@@ -1,0 +1,434 @@
+"""Benchmark of the Klein denoiser hot path on B200.
+
+One bench step = one full distilled text-to-image denoise at 1024x1024
+(512 text tokens + 64x64 image tokens, 16 shifted Euler steps, batch 1,
+random-init 5 + 28 block stack, bf16 weights and activations, fp32
+accumulation), through the public C-ABI entry point klein_denoise, inputs
+resident in HBM. `value` is Euler (denoise) steps per second summed over all
+ranks (replicas: each rank denoises its own image). The joint block at the
+same size (1.3916 TFLOP) is timed in the same run and reported as
+`joint_block`.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload t2i|edit|cfg2048] [--no-cpu-baseline]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "joint-block TFLOP/s & denoise steps/s at 1024² (frac of B200 BF16 peak)"
+DIM, MLP, LAT = 3072, 9216, 128
+
+WORKLOADS = {
+    # name: (batch, n_txt, img grid, refs, steps, cfg, distilled, description)
+    "t2i": (1, 512, (64, 64), (), 16, 1.0, True,
+            "distilled t2i denoise 1024x1024: 512 text + 64x64 image tokens (4608), 16 Euler steps, batch 1"),
+    "edit": (1, 512, (64, 64), ((64, 64),), 16, 1.0, True,
+             "distilled edit denoise 1024x1024 + one 1024x1024 reference: 512 + 4096 + 4096 tokens (8704), 16 steps"),
+    "cfg2048": (2, 560, (128, 128), (), 50, 3.5, False,
+                "base 2048x2048 denoise: 560 text + 128x128 image tokens (16944), 50 steps, CFG 3.5 as batch 2"),
+}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def block_gemm_flops_per_token():
+    return 2 * DIM * (3 * DIM + 2 * MLP) + 2 * (DIM + MLP) * DIM
+
+
+def attn_flops(rows):
+    return 4.0 * rows * rows * DIM
+
+
+def step_flops(batch, n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
+    """FLOPs of one denoiser call (multiply-add = 2): stage 1 per stream,
+    stage 2 over all tokens, input and output projections."""
+    n = n_txt + n_img + n_ref
+    f = 0.0
+    for r in (n_txt, n_img, n_ref):
+        if r:
+            f += n_stage1 * (r * block_gemm_flops_per_token() + attn_flops(r))
+    f += n_joint * (n * block_gemm_flops_per_token() + attn_flops(n))
+    f += 2.0 * (n_img + n_ref) * LAT * DIM + 2.0 * n_img * DIM * LAT
+    return batch * f
+
+
+def gemm_in_rows_per_step(n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
+    return n_stage1 * (n_txt + n_img + n_ref) + n_joint * (n_txt + n_img + n_ref)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.file,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def oracle_block_sample(n_txt=512, grid=(64, 64)):
+    """Times the CPU oracle's joint block at 512 + 64x64 tokens (one call)."""
+    import numpy as np
+    import klein_inputs as ki
+    import oracle as o
+    n_img = grid[0] * grid[1]
+    n = n_txt + n_img
+    w = ki.block_weights(0, "bench.oracle")
+    x = ki.tokens(1, "bench.oracle", 1, n)
+    mod = ki.modulation_vectors(1, "bench.oracle").astype(np.float64)
+    pos = o.positions(n_txt, grid)
+    modes = o.mode_of_rows(n_txt, n_img, 0)
+    t0 = time.perf_counter()
+    o.block(x, pos, modes, mod, w)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(wl):
+    batch, n_txt, grid, refs, steps, cfg, distilled, _ = WORKLOADS[wl]
+    n_img = grid[0] * grid[1]
+    n_ref = sum(h * w for h, w in refs)
+    t_block = oracle_block_sample()
+    f_block = 4608 * block_gemm_flops_per_token() + attn_flops(4608)
+    f_step = step_flops(batch, n_txt, n_img, n_ref)
+    t_step = t_block * f_step / f_block
+    return {"value": 1.0 / t_step, "unit": "denoise steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"one float64 oracle joint block at 512+4096 tokens timed once ({t_block:.2f} s, "
+                       f"{f_block / t_block / 1e9:.1f} GFLOP/s); steps/s extrapolated by FLOPs to one "
+                       f"{wl} denoise step ({f_step / 1e12:.2f} TFLOP)")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = args.workload
+    for _ in range(args.warmup):
+        oracle_block_sample(80, (8, 8))
+    times = [oracle_block_sample() for _ in range(args.steps)]
+    batch, n_txt, grid, refs, steps, cfg, distilled, desc = WORKLOADS[wl]
+    n_img = grid[0] * grid[1]
+    n_ref = sum(h * w for h, w in refs)
+    f_block = 4608 * block_gemm_flops_per_token() + attn_flops(4608)
+    f_step = step_flops(batch, n_txt, n_img, n_ref)
+    t_step = statistics.mean(times) * f_step / f_block
+    value = 1.0 / t_step
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "denoise steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": desc, "global_batch": batch, "seq_len": n_txt + n_img + n_ref,
+                       "parallelism": "none (CPU oracle, rank 0)"},
+            "cpu_baseline": {"value": value, "unit": "denoise steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": ("per step: one float64 oracle joint block at 512+4096 tokens, extrapolated "
+                                        "by FLOPs to one denoise step; warm-up steps use the 80+64-token block")},
+            "e2e": {"value": value, "unit": "denoise steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def random_block(g, dev):
+    import torch
+
+    def lin(o, i):
+        return (torch.randn(o, i, generator=g, device=dev) * (1.0 / math.sqrt(i))).to(torch.bfloat16)
+    w_out = torch.cat([lin(DIM, DIM), lin(DIM, MLP)], dim=1).contiguous()
+    return {"w_in": lin(3 * DIM + 2 * MLP, DIM), "w_out": w_out,
+            "q_norm": 1.0 + 0.1 * torch.randn(128, generator=g, device=dev),
+            "k_norm": 1.0 + 0.1 * torch.randn(128, generator=g, device=dev)}
+
+
+def random_model(dev, distilled, with_ref, seed=0):
+    import torch
+    g = torch.Generator(device=dev).manual_seed(seed)
+
+    def lin(o, i):
+        return (torch.randn(o, i, generator=g, device=dev) * (1.0 / math.sqrt(i))).to(torch.bfloat16)
+    t = {"stage1": {m: [random_block(g, dev) for _ in range(5)] for m in ("txt", "img")}}
+    t["stage1"]["ref"] = [random_block(g, dev) for _ in range(5)] if with_ref else []
+    t["joint"] = [random_block(g, dev) for _ in range(28)]
+    t.update({"img_in": lin(DIM, LAT), "ref_in": lin(DIM, LAT), "t_mlp1": lin(DIM, 256), "t_mlp2": lin(DIM, DIM),
+              "final_mod": lin(2 * DIM, DIM), "final_out": lin(LAT, DIM)})
+    for s in (1, 2):
+        for m in ("txt", "img", "ref"):
+            t[f"mod{s}.{m}"] = lin(3 * DIM, DIM)
+    if distilled:
+        t["tt_mlp1"], t["tt_mlp2"] = lin(DIM, 256), lin(DIM, DIM)
+    return t
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    import latent_flow_matching_joint_b200 as kb
+
+    batch, n_txt, grid, refs, steps, cfg, distilled, desc = WORKLOADS[args.workload]
+    seq = kb.make_seq(batch, n_txt, grid[0], grid[1], refs)
+    n_img, n_ref, n_total = kb.klein_seq_tokens(seq)
+    model_t = random_model(dev, distilled, bool(refs), seed=0)
+    model = kb.KleinModel(model_t)
+    g = torch.Generator(device=dev).manual_seed(1 + rank)
+    noise = torch.randn(n_img, LAT, generator=g, device=dev)
+    text = torch.randn(batch, n_txt, DIM, generator=g, device=dev).to(torch.bfloat16)
+    ref_lat = torch.randn(n_ref, LAT, generator=g, device=dev) if n_ref else None
+    lat = torch.empty_like(noise)
+    ws = torch.empty(kb.klein_stack_workspace_size(seq), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_image():
+        lat.copy_(noise)
+        kb.klein_denoise(model, lat, text, ref_lat, steps, cfg, seq, ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        one_image()
+    torch.cuda.synchronize()
+    rc, site, msg = kb.klein_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device error during warm-up: {msg}")
+
+    # ---- timed region: K full denoises, launch profiler on
+    launches0 = kb.klein_launch_count()
+    max_launches = (args.steps + 1) * steps * 400 + 100
+    kb.klein_profile_begin(max_launches)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clocks:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            one_image()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    prof = kb.klein_profile_end()
+    gpu_launches = kb.klein_launch_count() - launches0
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    rc, site, msg = kb.klein_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device error in the timed region: {msg}")
+    ms_per_image = ms / args.steps
+    value = world * steps * args.steps / (ms / 1e3)
+    f_step = step_flops(batch, n_txt, n_img, n_ref)
+    peaks = load_peaks()
+
+    # ---- dominant kernel roofline (in-projection GEMM, timed live above)
+    tot = sum(v[0] for v in prof.values())
+    top = max(prof, key=lambda k: prof[k][0])
+    gi_ms, gi_n = prof["gemm_in"]
+    gi_flops = batch * gemm_in_rows_per_step(n_txt, n_img, n_ref) * steps * args.steps * 2.0 * DIM * (3 * DIM + 2 * MLP)
+    gi_avg_ms = gi_ms / max(gi_n, 1)
+    achieved = gi_flops / (gi_ms / 1e3) / 1e12 if gi_ms > 0 else 0.0
+    roofline = {"kernel": "gemm_in (fused QKV + MLP-in, tcgen05)", "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
+                "traffic": None, "avg_launch_ms": gi_avg_ms, "launches": gi_n,
+                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
+
+    # ---- end to end through the public API with host buffers
+    noise_h = noise.cpu().pin_memory()
+    text_h = text.cpu().pin_memory()
+    ref_h = ref_lat.cpu().pin_memory() if n_ref else None
+    out_h = torch.empty_like(noise_h).pin_memory()
+    text_d = torch.empty_like(text)
+    ref_d = torch.empty_like(ref_lat) if n_ref else None
+
+    def e2e_image():
+        lat.copy_(noise_h, non_blocking=True)
+        text_d.copy_(text_h, non_blocking=True)
+        if n_ref:
+            ref_d.copy_(ref_h, non_blocking=True)
+        kb.klein_denoise(model, lat, text_d, ref_d, steps, cfg, seq, ws)
+        out_h.copy_(lat, non_blocking=True)
+
+    e2e_image()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_image()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    h2d = noise_h.numel() * 4 + text_h.numel() * 2 + (ref_h.numel() * 4 if n_ref else 0)
+    d2h = out_h.numel() * 4
+    e2e = {"value": world * steps * args.steps / (ms_e2e / 1e3), "unit": "denoise steps/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "note": "per bench step (one image): pinned host noise + text (+ reference) -> device, klein_denoise, "
+                   "final latents -> host"}
+
+    # ---- joint block at 512 + 4096 tokens (1024x1024 t2i), same run
+    jb = None
+    if args.workload == "t2i":
+        bw = model_t["joint"][0]
+        x = torch.randn(1, 4608, DIM, generator=g, device=dev).to(torch.bfloat16)
+        pos = torch.empty(4608, 4, device=dev)
+        kb.klein_positions(kb.make_seq(1, 512, 64, 64), pos)
+        mod = 0.5 * torch.randn(3, 3, DIM, generator=g, device=dev)
+        bws = torch.empty(kb.klein_block_workspace_size(1, 4608), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            kb.klein_block_forward(bw, x, 512, 4096, pos, mod, bws)
+        iters = 20
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            kb.klein_block_forward(bw, x, 512, 4096, pos, mod, bws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        bms = e0.elapsed_time(e1) / iters
+        bflops = 4608 * block_gemm_flops_per_token() + attn_flops(4608)
+        jb = {"ms": bms, "tflops": bflops / (bms / 1e3) / 1e12, "tokens_per_s": 4608 / (bms / 1e3),
+              "frac_of_peak": bflops / (bms / 1e3) / 1e12 / peaks["bf16"],
+              "peak": peaks["bf16"], "peak_source": f"{peaks['source']} bf16_tflops (burst, block timed alone)",
+              "algorithmic_tflop": bflops / 1e12}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "denoise steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_image, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": desc, "global_batch": world * batch, "seq_len": n_total, "parallelism": f"replicas x{world}",
+                   "euler_steps_per_bench_step": steps, "cfg": cfg, "distilled": distilled,
+                   "l2": "working set > L2 (11 GB of weights streamed per Euler step)",
+                   "weights": "random init N(0, 1/fan_in), bf16", "inputs": "N(0,1) noise and text embeddings"},
+        "tflops_per_gpu": f_step * steps * args.steps / (ms / 1e3) / 1e12,
+        "denoise_frac_of_peak": f_step * steps * args.steps / (ms / 1e3) / 1e12 / peaks["bf16_sustained"],
+        "roofline": roofline,
+        "kernels": {k: {"ms": v[0], "launches": v[1], "share": (v[0] / tot if tot else 0.0)} for k, v in prof.items()},
+        "top_kernel": top,
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+        "clocks": clocks.summary(),
+    }
+    if jb:
+        line["joint_block"] = jb
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del model
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=tuple(WORKLOADS), default="t2i")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,279 @@
+/*
+ * klein.h - C ABI of the B200 (sm_100a) implementation of the FLUX.3 Image
+ * Klein denoiser hot path: the joint transformer block over the concatenated
+ * [text | noisy image | reference] token sequence, run inside the shifted
+ * flow-matching Euler loop.
+ *
+ * Sources (cited by page and section):
+ *   [blog]   "FLUX.3 Image Klein Is Now Available in Diffusers", section
+ *            "Speed, architecture, and how the tokens move" (two stages,
+ *            block shape, modulation by stream, RoPE axes).
+ *   [blogzh] its Chinese translation: block pseudo-code and RoPE table.
+ *   [guide]  "How to Run FLUX 3 Image Klein Locally": "The latent space and
+ *            the VAE", "Inside the transformer", "The denoise loop", "What
+ *            step distillation removed", "Why dropping CFG halves the compute".
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are caller-owned CUDA device memory; the
+ *     library borrows them for the duration of the asynchronous work it
+ *     enqueues and never frees them. "host" pointers are read or written
+ *     before the call returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).
+ *   - Argument errors are detected synchronously and return a negative
+ *     klein_status with nothing enqueued; klein_last_error() then returns a
+ *     message (thread-local, valid until the next call on that thread).
+ *   - A failed kernel launch returns KLEIN_ERR_CUDA. A device-side wait that
+ *     gave up (no progress for the wait limit) is recorded on the device and
+ *     reported by klein_device_status() as KLEIN_ERR_TIMEOUT.
+ *   - Device pointers must be 16-byte aligned. The model width is fixed at
+ *     KLEIN_DIM = 3072, 24 heads of 128.
+ *   - bf16 = IEEE bfloat16 stored as uint16; all matrices are row-major.
+ *   - Nothing is thrown across the ABI; no call allocates device memory:
+ *     scratch comes from the caller's workspace.
+ */
+#ifndef KLEIN_H
+#define KLEIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KLEIN_DIM 3072
+#define KLEIN_HEADS 24
+#define KLEIN_HEAD_DIM 128
+#define KLEIN_MLP_HIDDEN 9216
+#define KLEIN_LATENT_CH 128
+#define KLEIN_MAX_REFS 10
+#define KLEIN_IN_COLS (3 * KLEIN_DIM + 2 * KLEIN_MLP_HIDDEN)  /* 27648 */
+#define KLEIN_OUT_K (KLEIN_DIM + KLEIN_MLP_HIDDEN)            /* 12288 */
+
+typedef enum {
+  KLEIN_OK = 0,
+  KLEIN_ERR_INVALID_ARG = -1,
+  KLEIN_ERR_SHAPE = -2,
+  KLEIN_ERR_ALIGN = -3,
+  KLEIN_ERR_WORKSPACE = -4,
+  KLEIN_ERR_CUDA = -5,
+  KLEIN_ERR_TIMEOUT = -6,
+  KLEIN_ERR_UNSUPPORTED = -7
+} klein_status;
+
+/* Message describing the last error on this thread ("" if none). */
+const char* klein_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+int klein_version(void);
+
+/* Number of kernels this library has launched in this process (host-side
+ * counter over every entry point; for launch accounting in benchmarks). */
+long long klein_launch_count(void);
+
+/* Reads and clears the device error word on the current device (blocking:
+ * synchronises the device). Returns KLEIN_OK, KLEIN_ERR_TIMEOUT when a
+ * bounded wait gave up, KLEIN_ERR_CUDA on a CUDA error. `site` (may be NULL)
+ * receives the code of the wait that gave up. */
+int klein_device_status(unsigned* site);
+
+/* Sets the bound (nanoseconds) of every device-side wait; default 2 s. */
+int klein_set_wait_limit_ns(unsigned long long ns);
+
+/* Enqueues a probe kernel that waits, with the given bound, on a barrier
+ * that nothing arrives on. It must end by recording KLEIN_ERR_TIMEOUT, which
+ * klein_device_status() then returns. Tests the wait bound, nothing else. */
+int klein_wait_probe(unsigned long long limit_ns, void* stream);
+
+/* Launch profiler. While running, the library records a pair of CUDA
+ * events on the launching stream around each kernel launch of the path and
+ * tags it with its kind (index into the arrays below):
+ *   0 modulated LayerNorm, 1 in-projection GEMM (QKV + MLP-in, fused
+ *   epilogue), 2 attention, 3 out-projection GEMM (gated residual),
+ *   4 timestep embedding + modulation, 5 input / output projections,
+ *   6 Euler update, 7 other.
+ * klein_profile_begin(max_launches) creates the events (host-side
+ * resources; no device memory); klein_profile_end synchronises, writes the
+ * summed milliseconds and launch counts per kind (arrays of
+ * KLEIN_PROF_KINDS, either may be NULL) and releases the events. Returns
+ * KLEIN_ERR_WORKSPACE if more launches happened than max_launches (those
+ * were not timed). Not thread-safe; one profile at a time. */
+#define KLEIN_PROF_KINDS 8
+int klein_profile_begin(int max_launches);
+int klein_profile_end(double* ms, int* launches);
+
+/* ------------------------------------------------------------------ sequence */
+
+/* Token layout of one denoiser call: rows [0, n_txt) text, then the image
+ * grid img_h x img_w scanned row-major, then each reference grid in order
+ * ([blog]: the sequence is [text | image | reference]). A 1024x1024 image
+ * is a 64 x 64 grid of 4096 tokens ([guide] "The latent space and the VAE"). */
+typedef struct {
+  int batch;                    /* B: 1, or 2 for guidance (cond, uncond) */
+  int n_txt;                    /* text tokens per batch item (>= 1) */
+  int img_h, img_w;             /* image token grid */
+  int n_refs;                   /* reference images, 0..KLEIN_MAX_REFS */
+  int ref_h[KLEIN_MAX_REFS];    /* reference token grids */
+  int ref_w[KLEIN_MAX_REFS];
+} klein_seq;
+
+/* Token counts of `seq`; any output pointer may be NULL. */
+int klein_seq_tokens(const klein_seq* seq, int* n_img, int* n_ref, int* n_total);
+
+/* Text length padded to a multiple of 80 ([blog]; [guide] "The text
+ * encoder"). A helper: the kernels accept any n_txt. Returns -1 if n < 0. */
+int klein_pad_text_len(int n);
+
+/* Shifted sigma schedule ([guide] "The denoise loop"): `steps` levels evenly
+ * spaced from 1 down to 1/steps, each mapped to s*sigma/(1+(s-1)*sigma),
+ * then a final 0. sigmas: host, steps + 1 floats. Computed in double. */
+int klein_sigma_schedule(int steps, float shift, float* sigmas);
+
+/* (t, h, w, l) per token ([blogzh] RoPE table; Chinese summary page for
+ * the negative reference offset): text i -> (0,0,0,i); image token (r,c)
+ * -> (0,r,c,0); token (r,c) of reference k -> (0,r,c,-(k+1)).
+ * pos: device, [n_total][4] float. */
+int klein_positions(const klein_seq* seq, float* pos, void* stream);
+
+/* ------------------------------------------------------------------ block */
+
+/* Weights of one block (device, borrowed):
+ *   w_in   bf16 [27648][3072]: output rows q(3072) | k(3072) | v(3072) |
+ *          gate(9216) | up(9216); the SwiGLU hidden is silu(gate) * up.
+ *   w_out  bf16 [3072][12288]: input columns attention (3072, the attention
+ *          output projection) | MLP down (9216).
+ *   q_norm, k_norm  float [128]: QK-RMSNorm weights shared by all heads. */
+typedef struct {
+  const void* w_in;
+  const void* w_out;
+  const float* q_norm;
+  const float* k_norm;
+} klein_block_weights;
+
+/* Workspace bytes for klein_block_forward on `rows` rows of `batch` items. */
+size_t klein_block_workspace_size(int batch, int rows);
+
+/* One block, in place on rows [row0, row0 + rows) of every batch item of x
+ * ([blogzh] block pseudo-code; [blog]; [guide] "Inside the transformer"):
+ * no-affine LayerNorm modulated per stream (text rows use mode 0, image
+ * rows mode 1, reference rows mode 2, by global row index against n_txt
+ * and n_txt + n_img); q, k, v and the SwiGLU MLP from that one normalised
+ * input; RMSNorm + 4-axis RoPE on q and k; softmax attention among the
+ * `rows` rows only, no mask; x += gate * (attention out-projection + MLP).
+ * A joint block passes row0 = 0, rows = n_total; a stage-1 block passes one
+ * stream's row range (each stream attends only to itself).
+ *   x        device bf16 [batch][n_total][3072], updated in place
+ *   pos      device float [n_total][4] (klein_positions)
+ *   mod      device float [3 modes][3 (shift, scale, gate)][3072]
+ *   ws       device workspace, >= klein_block_workspace_size(batch, rows)
+ * Errors: KLEIN_ERR_SHAPE if rows < 1 or the range leaves [0, n_total). */
+int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_total, int row0, int rows,
+                        int n_txt, int n_img, const float* pos, const float* mod, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* ------------------------------------------------------------------ model */
+
+/* All weights of a stack (device, borrowed; bf16 [out][in] unless noted).
+ * Model: n_stage1 = 5 per-stream blocks and n_joint = 28 joint blocks
+ * ([blog]; [guide] "Inside the transformer"); smaller counts are accepted. */
+typedef struct {
+  int n_stage1;
+  int n_joint;
+  const klein_block_weights* stage1[3];  /* per stream (txt, img, ref): n_stage1 each */
+  const klein_block_weights* joint;      /* n_joint */
+  const void* img_in;      /* [3072][128] image latent projection */
+  const void* ref_in;      /* [3072][128] reference latent projection (may be NULL without refs) */
+  const void* t_mlp1;      /* [3072][256] timestep embedder, layer 1 */
+  const void* t_mlp2;      /* [3072][3072] layer 2 */
+  const void* tt_mlp1;     /* target-level embedder of the distilled model, or NULL (base) */
+  const void* tt_mlp2;
+  const void* mod[2][3];   /* [9216][3072] per stage (1, 2) and stream: (shift, scale, gate) */
+  const void* final_mod;   /* [6144][3072] final (shift, scale) */
+  const void* final_out;   /* [128][3072] output projection to latent channels */
+} klein_model_desc;
+
+typedef struct klein_model klein_model;
+
+/* Copies the descriptor (not the weights) into a new handle. */
+int klein_model_create(klein_model** out, const klein_model_desc* desc);
+void klein_model_destroy(klein_model* m);
+
+/* Workspace bytes for klein_stack_forward / klein_denoise on `seq`. */
+size_t klein_stack_workspace_size(const klein_seq* seq);
+
+/* One denoiser call ([blog]; [guide] "Inside the transformer", "What step
+ * distillation removed"): modulation from the timestep embedding (image
+ * rows at sigma, text and reference rows at 0, plus the target-level
+ * embedding of sigma_next on every stream when the model is distilled);
+ * image and reference latents projected to 3072; stage 1 runs each stream's
+ * own blocks over its own rows; stage 2 runs the joint blocks over
+ * [text | image | reference]; the image rows then pass the final modulated
+ * LayerNorm and projection to 128 channels.
+ *   latents  device float [n_img][128], shared by the batch
+ *   text     device bf16 [batch][n_txt][3072]
+ *   refs     device float [n_ref][128] or NULL when seq->n_refs == 0
+ *   v_out    device float [batch][n_img][128]
+ *   ws       device workspace >= klein_stack_workspace_size(seq) */
+int klein_stack_forward(const klein_model* m, const float* latents, const void* text, const float* refs,
+                        float sigma, float sigma_next, const klein_seq* seq, float* v_out, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* Flow-matching Euler sampler ([guide] "The denoise loop", "Why dropping CFG
+ * halves the compute"): from sigma = 1 over klein_sigma_schedule(steps,
+ * shift), each step runs klein_stack_forward and moves the latents by
+ * (sigma_next - sigma) * v. cfg > 1 needs seq->batch == 2 (text = cond then
+ * uncond) and uses v = v_u + cfg (v_c - v_u); otherwise seq->batch == 1.
+ *   latents  device float [n_img][128]: in = noise, out = the final latents
+ *   x0_out   device float [n_img][128] or NULL: the last step's x0 preview */
+int klein_denoise(const klein_model* m, float* latents, const void* text, const float* refs, int steps,
+                  float cfg, float shift, const klein_seq* seq, float* x0_out, void* ws, size_t ws_bytes,
+                  void* stream);
+
+/* ------------------------------------------------------------------ single ops
+ * The kernels of the path, exposed one by one for parity tests and the
+ * memory-bound benchmarks. Same conventions as above. */
+
+/* h = modulated LayerNorm of rows [row0, row0 + rows) of x (mode by global
+ * row as in klein_block_forward). mod: [3][>=2][3072] with per-mode stride
+ * mod_stride floats; single_mode != 0 applies mod[0] to every row.
+ * x: bf16 [batch][n_total][3072]; h: bf16 [batch][rows][3072]. */
+int klein_op_modln(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
+                   const float* mod, long long mod_stride, int single_mode, void* h, void* stream);
+
+/* cos/sin table [rows][64] (float2) of the 4-axis RoPE, theta = base. */
+int klein_op_rope_table(const float* pos, int rows, float theta, void* table, void* stream);
+
+/* out = RoPE(in) for bf16 [rows][heads][128] using a table from
+ * klein_op_rope_table (in and out may alias). */
+int klein_op_rope(const void* in, void* out, const void* table, int rows, int heads, void* stream);
+
+/* x += dsigma * v with v = v_cond, or v_u + g (v_c - v_u) when v_uncond is
+ * not NULL; x0_out (optional) = x - sigma * v, from x before the update.
+ * float arrays of n elements, n a multiple of 4. */
+int klein_op_euler(float* x, const float* v_cond, const float* v_uncond, long long n, float dsigma, float g,
+                   float* x0_out, float sigma, void* stream);
+
+/* C[M][N] (float) = A[M][K] * B[N][K]^T, bf16 operands, tcgen05 tensor cores.
+ * M >= 1, N a multiple of 128, K a multiple of 64. */
+int klein_op_gemm(const void* a, const void* b, float* c, int m, int n, int k, void* stream);
+
+/* Softmax attention per (batch, head) over `rows` rows, scale 1/sqrt(128),
+ * no mask. q, k: bf16 [batch][24][rows_pad][128]; vt: bf16
+ * [batch][24][128][rows_pad] (v transposed); out: bf16 [batch][rows][out_ld]
+ * with head h in columns h*128..h*128+127. rows_pad >= rows, a multiple of 8. */
+int klein_op_attention(const void* q, const void* k, const void* vt, int batch, int rows, int rows_pad,
+                       void* out, long long out_ld, void* stream);
+
+/* Per-stage, per-stream modulation and the final (shift, scale) of one
+ * denoiser call (see klein_stack_forward). mod_out: device float
+ * [2][3][3][3072]; final_out: device float [2][3072]; ws: device,
+ * >= 24576 floats (8 x 3072). */
+int klein_op_time_mod(const klein_model* m, float sigma, float sigma_next, int with_ref, float* mod_out,
+                      float* final_out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLEIN_H */

@@ -1,0 +1,347 @@
+// Persistent tcgen05 GEMM, C = A * B^T, bf16 operands, fp32 accumulation in
+// tensor memory, fed by TMA, with the block's fused epilogues.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 per stage
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2..5  epilogue: one accumulator row per thread (TMEM lane quarter
+//               = warp % 4), two accumulator buffers so that the epilogue of
+//               tile i overlaps the main loop of tile i+1.
+// Tiles are visited M-fastest so the CTAs in flight share B tiles in L2.
+//
+// Epilogues (FLUX.3 Klein block, Diffusers release blog "Speed,
+// architecture, and how the tokens move", and its Chinese translation's
+// block pseudo-code):
+//   kEpiQKV   in-projection: q and k are RMS-normalised per head and rotated
+//             by the 4-axis RoPE, v is stored transposed for the attention
+//             kernel, and the paired gate|up tiles leave silu(gate) * up.
+//   kEpiResid out-projection: x += gate[mode(row)] * (attn + mlp).
+#include "common.cuh"
+#include "internal.h"
+
+namespace klein {
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStageA = 128 * 64 * 2;
+  static constexpr int kStageB = BN * 64 * 2;
+  static constexpr int kStage = kStageA + kStageB;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kTileBytes = kStages * kStage;
+  static constexpr int kSmem = kTileBytes + 1024 + 256;
+  static constexpr uint32_t kTmemCols = 2 * BN;
+  static constexpr int kThreads = 192;
+};
+
+static constexpr float kRmsEps = 1e-6f;
+
+__device__ __forceinline__ void store16(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
+}
+
+// ---- epilogues: one thread = one accumulator row; taddr = lane quarter base
+
+template <int BN>
+__device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, bool f32) {
+  const bool valid = r < g.rows;
+  float v[32];
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    tmem_ld32(taddr + 32 * c, v);
+    if (!valid) continue;
+    const int col = n_idx * BN + 32 * c;
+    const int copies = g.replicate > 1 ? g.replicate : 1;
+    for (int rep = 0; rep < copies; ++rep) {
+      const int bb = g.replicate > 1 ? rep : b;
+      const long long orow = (long long)bb * g.out_bstride + g.out_row0 + r;
+      if (f32) {
+        float* o = reinterpret_cast<float*>(g.out) + orow * g.out_ld + col;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + orow * g.out_ld + col;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          store16(o + i, pack_bf16(v[i], v[i + 1]), pack_bf16(v[i + 2], v[i + 3]), pack_bf16(v[i + 4], v[i + 5]),
+                  pack_bf16(v[i + 6], v[i + 7]));
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
+  const bool valid = r < g.rows;
+  float v[32];
+  if (n_idx < g.b_split) {
+    const int which = n_idx / 12;            // 0 q, 1 k, 2 v
+    const int head0 = (n_idx % 12) * 2;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      const int head = head0 + hh;
+      const uint32_t tcol = taddr + hh * 128;
+      const long long bh = (long long)b * kHeads + head;
+      if (which == 2) {
+        __nv_bfloat16* dst = g.vt + bh * kHeadDim * g.rows_pad + r;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tcol + 32 * c, v);
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dst[(long long)(32 * c + i) * g.rows_pad] = __float2bfloat16_rn(v[i]);
+          }
+        }
+        continue;
+      }
+      const float* w = which == 0 ? g.q_norm : g.k_norm;
+      __nv_bfloat16* dst = (which == 0 ? g.q : g.k) + (bh * g.rows_pad + r) * kHeadDim;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tcol + 32 * c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+      const float rs = rsqrtf(ss * (1.0f / kHeadDim) + kRmsEps);
+      const float2* rope = g.rope + (long long)(valid ? r : 0) * kPairs;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tcol + 32 * c, v);
+        if (!valid) continue;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int d = 32 * c + i;
+          const float y0 = v[i] * rs * __ldg(w + d);
+          const float y1 = v[i + 1] * rs * __ldg(w + d + 1);
+          const float2 cs = rope[d >> 1];
+          pk[i >> 1] = pack_bf16(y0 * cs.x - y1 * cs.y, y0 * cs.y + y1 * cs.x);
+        }
+        __nv_bfloat16* o = dst + 32 * c;
+        store16(o, pk[0], pk[1], pk[2], pk[3]);
+        store16(o + 8, pk[4], pk[5], pk[6], pk[7]);
+        store16(o + 16, pk[8], pk[9], pk[10], pk[11]);
+        store16(o + 24, pk[12], pk[13], pk[14], pk[15]);
+      }
+    }
+  } else {
+    const int chunk = n_idx - g.b_split;     // 128 hidden units: gate cols 0..127, up cols 128..255
+    __nv_bfloat16* dst = g.a_out + ((long long)b * g.rows + r) * kOutK + kDim + chunk * 128;
+    float u[32];
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(taddr + 32 * c, v);
+      tmem_ld32(taddr + 128 + 32 * c, u);
+      if (!valid) continue;
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16(silu(v[i]) * u[i], silu(v[i + 1]) * u[i + 1]);
+      __nv_bfloat16* o = dst + 32 * c;
+      store16(o, pk[0], pk[1], pk[2], pk[3]);
+      store16(o + 8, pk[4], pk[5], pk[6], pk[7]);
+      store16(o + 16, pk[8], pk[9], pk[10], pk[11]);
+      store16(o + 24, pk[12], pk[13], pk[14], pk[15]);
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
+  const bool valid = r < g.rows;
+  const int grow = g.x_row0 + r;
+  const int mode = mode_of_row(grow, g.n_txt, g.n_img);
+  const float* gate = g.mod + (long long)mode * 3 * kDim + 2 * kDim + n_idx * BN;
+  __nv_bfloat16* xr = g.x + ((long long)b * g.x_bstride + grow) * kDim + n_idx * BN;
+  float v[32];
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    tmem_ld32(taddr + 32 * c, v);
+    if (!valid) continue;
+    __nv_bfloat16* p = xr + 32 * c;
+    const float* gt = gate + 32 * c;
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 raw = *reinterpret_cast<const uint4*>(p + i);
+      float2 a0 = unpack_bf16(raw.x), a1 = unpack_bf16(raw.y), a2 = unpack_bf16(raw.z), a3 = unpack_bf16(raw.w);
+      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gt + i));
+      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gt + i + 4));
+      raw.x = pack_bf16(fmaf(g0.x, v[i + 0], a0.x), fmaf(g0.y, v[i + 1], a0.y));
+      raw.y = pack_bf16(fmaf(g0.z, v[i + 2], a1.x), fmaf(g0.w, v[i + 3], a1.y));
+      raw.z = pack_bf16(fmaf(g1.x, v[i + 4], a2.x), fmaf(g1.y, v[i + 5], a2.y));
+      raw.w = pack_bf16(fmaf(g1.z, v[i + 6], a3.x), fmaf(g1.w, v[i + 7], a3.y));
+      *reinterpret_cast<uint4*>(p + i) = raw;
+    }
+  }
+}
+
+// ---- the kernel
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const GemmArgs g) {
+  using Cfg = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kTileBytes);
+  uint64_t* empty = full + Cfg::kStages;
+  uint64_t* acc_full = empty + Cfg::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = g.batch * g.m_tiles_per_b;
+  const int total = m_tiles * g.n_tiles;
+  constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const int m_idx = tile % m_tiles;
+        const int n_idx = tile / m_tiles;
+        const int b = m_idx / g.m_tiles_per_b;
+        const int row0 = (m_idx % g.m_tiles_per_b) * 128;
+        int brow0, brow1;
+        if (EPI == kEpiQKV && n_idx >= g.b_split) {
+          const int chunk = n_idx - g.b_split;
+          brow0 = 3 * kDim + chunk * 128;
+          brow1 = 3 * kDim + kMlp + chunk * 128;
+        } else {
+          brow0 = n_idx * BN;
+          brow1 = brow0 + 128;
+        }
+        bool ok = true;
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, 0x101)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], Cfg::kStage);
+          uint8_t* sa = smem + stage * Cfg::kStage;
+          uint8_t* sb = sa + Cfg::kStageA;
+          tma_load_3d(sa, &map_a, &full[stage], kb * 64, row0, b);
+          tma_load_2d(sb, &map_b, &full[stage], kb * 64, brow0);
+          if (BN == 256) tma_load_2d(sb + 128 * 128, &map_b, &full[stage], kb * 64, brow1);
+          if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, 0x102)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, 0x103)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * Cfg::kStage);
+          const uint32_t b0 = a0 + Cfg::kStageA;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, (kb | k) != 0);
+          umma_commit(&empty[stage]);
+          if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int rloc = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int m_idx = tile % m_tiles;
+      const int n_idx = tile / m_tiles;
+      const int b = m_idx / g.m_tiles_per_b;
+      const int r = (m_idx % g.m_tiles_per_b) * 128 + rloc;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&acc_full[acc], acc_phase, 0x104)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (EPI == kEpiF32) epi_store<BN>(taddr, g, b, r, n_idx, true);
+      else if (EPI == kEpiBF16) epi_store<BN>(taddr, g, b, r, n_idx, false);
+      else if (EPI == kEpiQKV) epi_qkv(taddr, g, b, r, n_idx);
+      else epi_resid<BN>(taddr, g, b, r, n_idx);
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int BN, int EPI>
+static int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
+  using Cfg = GemmCfg<BN>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+        cudaSuccess)
+      return -1;
+    configured = true;
+  }
+  const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
+  if (total <= 0) return 0;
+  const int grid = total < num_sms() ? total : num_sms();
+  gemm_kernel<BN, EPI><<<grid, Cfg::kThreads, Cfg::kSmem, s>>>(ma, mb, g);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_gemm(int bn, int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                cudaStream_t s) {
+  if (bn == 256) {
+    switch (epi) {
+      case kEpiF32: return launch_one<256, kEpiF32>(ma, mb, g, s);
+      case kEpiBF16: return launch_one<256, kEpiBF16>(ma, mb, g, s);
+      case kEpiQKV: return launch_one<256, kEpiQKV>(ma, mb, g, s);
+      case kEpiResid: return launch_one<256, kEpiResid>(ma, mb, g, s);
+    }
+  } else if (bn == 128) {
+    switch (epi) {
+      case kEpiF32: return launch_one<128, kEpiF32>(ma, mb, g, s);
+      case kEpiBF16: return launch_one<128, kEpiBF16>(ma, mb, g, s);
+    }
+  }
+  return -2;
+}
+
+}  // namespace klein

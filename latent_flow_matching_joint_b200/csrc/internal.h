@@ -1,0 +1,117 @@
+// Internal (C++) interface between the Klein kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace klein {
+
+// ------------------------------------------------------------------ TMA maps
+
+// 2-D bf16 tensor map over a row-major [outer][inner] matrix with row pitch
+// `row_bytes`; box = box_inner x box_outer elements, 128-byte swizzle.
+int make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                uint32_t box_inner, uint32_t box_outer);
+// 3-D bf16 tensor map over [d2][d1][d0] with byte strides s1 (d1) and s2 (d2).
+int make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                uint64_t s2, uint32_t box0, uint32_t box1);
+
+// ------------------------------------------------------------------ GEMM
+
+enum EpiKind : int {
+  kEpiF32 = 0,    // out fp32 = acc
+  kEpiBF16 = 1,   // out bf16 = acc (optionally replicated over batch copies)
+  kEpiQKV = 2,    // fused in-projection: RMSNorm + RoPE on q/k, v transposed, SwiGLU
+  kEpiResid = 3,  // x += gate[mode(row)] * acc
+};
+
+struct GemmArgs {
+  int batch;          // batch items of A (3-D map depth)
+  int rows;           // valid rows of A per batch item (M)
+  int m_tiles_per_b;  // ceil(rows / 128)
+  int n_tiles;        // N / BN
+  int k_blocks;       // K / 64
+  int b_split;        // kEpiQKV: the N-tile where the paired gate|up tiles begin
+  // kEpiF32 / kEpiBF16: out[(b * out_bstride + out_row0 + r) * out_ld + n]
+  void* out;
+  long long out_ld;
+  long long out_bstride;
+  int out_row0;
+  int replicate;      // >1: A has one batch item; write its rows into this many batch copies
+  // kEpiQKV
+  __nv_bfloat16* q;   // [batch][24][rows_pad][128]
+  __nv_bfloat16* k;   // [batch][24][rows_pad][128]
+  __nv_bfloat16* vt;  // [batch][24][128][rows_pad]
+  __nv_bfloat16* a_out;  // [batch][rows][12288]; SwiGLU goes to columns 3072..
+  const float* q_norm;
+  const float* k_norm;
+  const float2* rope;  // [rows][64] (cos, sin)
+  int rows_pad;
+  // kEpiResid
+  __nv_bfloat16* x;   // [batch][x_bstride rows][3072]
+  long long x_bstride;
+  int x_row0;
+  const float* mod;   // [3 modes][3][3072] (shift, scale, gate)
+  int n_txt, n_img;
+};
+
+// C[M,N] = A[M,K] * B[N,K]^T with epilogue `epi`; bn = 128 or 256.
+int launch_gemm(int bn, int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
+                cudaStream_t stream);
+
+// ------------------------------------------------------------------ attention
+
+struct AttnArgs {
+  int batch, heads, rows, rows_pad;
+  __nv_bfloat16* out;   // [batch][rows][out_ld], head h at columns h*128..
+  long long out_ld;
+  float scale_log2;     // log2(e) / sqrt(128)
+};
+
+int launch_attention(const CUtensorMap& map_q, const CUtensorMap& map_k, const CUtensorMap& map_vt,
+                     const AttnArgs& args, cudaStream_t stream);
+
+// ------------------------------------------------------------------ memory-bound kernels
+
+int launch_modln(const __nv_bfloat16* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
+                 int n_txt, int n_img, const float* mod, long long mod_mode_stride, int single_mode,
+                 cudaStream_t stream);
+int launch_rope_table(const float* pos, float2* table, int rows, float theta, cudaStream_t stream);
+int launch_rope_apply(const __nv_bfloat16* in, __nv_bfloat16* out, const float2* table, int rows, int heads,
+                      cudaStream_t stream);
+int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, const int* ref_h,
+                     const int* ref_w, cudaStream_t stream);
+int launch_euler(float* x, const float* v_cond, const float* v_uncond, long long n, float dsigma, float g,
+                 float* x0_out, float sigma, cudaStream_t stream);
+int launch_to_bf16(const float* in, __nv_bfloat16* out, long long n, cudaStream_t stream);
+int launch_copy_rows(const __nv_bfloat16* src, long long src_bstride, __nv_bfloat16* dst, long long dst_bstride,
+                     int dst_row0, int batch, int rows, int src_batches, cudaStream_t stream);
+
+// Timestep embedding + modulation (a2).
+struct TimeModArgs {
+  const __nv_bfloat16* t_mlp1;  // [3072][256]
+  const __nv_bfloat16* t_mlp2;  // [3072][3072]
+  const __nv_bfloat16* tt_mlp1; // distilled target-time embedder, or null
+  const __nv_bfloat16* tt_mlp2;
+  const __nv_bfloat16* mod[2][3];  // [9216][3072]
+  const __nv_bfloat16* final_mod;  // [6144][3072]
+  float sigma, sigma_next;
+  int with_ref;
+  float* scratch;       // >= 8 * 3072 floats
+  float* mod_out;       // [2][3][3][3072]
+  float* final_out;     // [2][3072]
+};
+int launch_time_mod(const TimeModArgs& a, cudaStream_t stream);
+int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_vec, long long x_stride,
+                float* y, long long y_stride, int act_in_silu, const float* add, cudaStream_t stream);
+
+int launch_wait_probe(unsigned long long limit_ns, cudaStream_t stream);
+int num_sms();
+
+// Host-side count of kernels launched by this library (all entry points).
+void note_launch();
+
+}  // namespace klein

@@ -1,0 +1,404 @@
+// HBM-bound and small kernels of the Klein hot path: modulated LayerNorm,
+// RoPE table and standalone rotation, token positions, Euler/CFG update,
+// bf16 conversion, timestep embedding and the modulation GEMVs.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace klein {
+
+// ------------------------------------------------------------------ modLN
+// Parameter-free LayerNorm of each row, then (1 + scale[m]) * xhat + shift[m]
+// with m the row's stream (Diffusers release blog for FLUX.3 Klein, "Speed,
+// architecture, and how the tokens move": no learned affine; text and
+// reference rows take the t = 0 modulation, image rows the current t).
+// One warp per row; 12 x 16-byte loads per lane; fp32 statistics.
+
+__global__ void __launch_bounds__(256, 2) modln_kernel(const __nv_bfloat16* __restrict__ x, long long x_bstride,
+                                                    int x_row0, __nv_bfloat16* __restrict__ h, int batch,
+                                                    int rows, int n_txt, int n_img,
+                                                    const float* __restrict__ mod, long long mod_stride,
+                                                    int single_mode) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= batch * rows) return;
+  const int b = warp / rows;
+  const int i = warp % rows;
+  const int grow = x_row0 + i;
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)b * x_bstride + grow) * kDim);
+  uint4* dst = reinterpret_cast<uint4*>(h + ((long long)b * rows + i) * kDim);
+  constexpr int kVec = kDim / 8 / 32;  // 12 uint4 per lane, kept packed
+  uint4 raw[kVec];
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) raw[t] = __ldcs(src + lane + 32 * t);
+  float sum = 0.f;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const uint32_t w4[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 e = unpack_bf16(w4[q]);
+      sum += e.x + e.y;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum * (1.0f / kDim);
+  float sq = 0.f;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const uint32_t w4[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 e = unpack_bf16(w4[q]);
+      const float d0 = e.x - mean, d1 = e.y - mean;
+      sq = fmaf(d0, d0, fmaf(d1, d1, sq));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = rsqrtf(sq * (1.0f / kDim) + 1e-6f);
+  const int m = single_mode ? 0 : mode_of_row(grow, n_txt, n_img);
+  const float* shift = mod + m * mod_stride;
+  const float* scale = shift + kDim;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const int col = 8 * (lane + 32 * t);
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(scale + col));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(scale + col + 4));
+    const float4 h0 = __ldg(reinterpret_cast<const float4*>(shift + col));
+    const float4 h1 = __ldg(reinterpret_cast<const float4*>(shift + col + 4));
+    const float2 e0 = unpack_bf16(raw[t].x), e1 = unpack_bf16(raw[t].y);
+    const float2 e2 = unpack_bf16(raw[t].z), e3 = unpack_bf16(raw[t].w);
+    uint4 o;
+    o.x = pack_bf16(fmaf((e0.x - mean) * rstd, 1.f + s0.x, h0.x), fmaf((e0.y - mean) * rstd, 1.f + s0.y, h0.y));
+    o.y = pack_bf16(fmaf((e1.x - mean) * rstd, 1.f + s0.z, h0.z), fmaf((e1.y - mean) * rstd, 1.f + s0.w, h0.w));
+    o.z = pack_bf16(fmaf((e2.x - mean) * rstd, 1.f + s1.x, h1.x), fmaf((e2.y - mean) * rstd, 1.f + s1.y, h1.y));
+    o.w = pack_bf16(fmaf((e3.x - mean) * rstd, 1.f + s1.z, h1.z), fmaf((e3.y - mean) * rstd, 1.f + s1.w, h1.w));
+    dst[lane + 32 * t] = o;
+  }
+}
+
+int launch_modln(const __nv_bfloat16* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
+                 int n_txt, int n_img, const float* mod, long long mod_stride, int single_mode, cudaStream_t s) {
+  const long long warps = (long long)batch * rows;
+  if (warps <= 0) return 0;
+  const int blocks = (int)((warps + 7) / 8);
+  modln_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, h, batch, rows, n_txt, n_img, mod, mod_stride,
+                                      single_mode);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ RoPE
+// Four axes (t, h, w, l), 32 head dims each (blog, RoPE paragraph); pair p =
+// 16 * axis + j covers dims (2p, 2p+1) and turns by pos[axis] * theta^(-j/16).
+// The table is built in double precision once per sequence.
+
+__global__ void rope_table_kernel(const float* __restrict__ pos, float2* __restrict__ table, int rows,
+                                  double theta) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * kPairs) return;
+  const int r = idx / kPairs;
+  const int p = idx % kPairs;
+  const int axis = p >> 4;
+  const int j = p & 15;
+  const double freq = pow(theta, -static_cast<double>(j) / 16.0);
+  const double ang = static_cast<double>(pos[r * 4 + axis]) * freq;
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  table[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+}
+
+int launch_rope_table(const float* pos, float2* table, int rows, float theta, cudaStream_t s) {
+  const int n = rows * kPairs;
+  if (n <= 0) return 0;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(pos, table, rows, static_cast<double>(theta));
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// Standalone rotation of [rows][heads][128] bf16 (the same arithmetic as the
+// in-projection epilogue). One thread per 8 elements (4 pairs).
+__global__ void rope_apply_kernel(const uint4* __restrict__ in, uint4* __restrict__ out,
+                                  const float2* __restrict__ table, int rows, int heads) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long total = (long long)rows * heads * (kHeadDim / 8);
+  if (idx >= total) return;
+  const int chunk = static_cast<int>(idx % (kHeadDim / 8));
+  const int r = static_cast<int>(idx / ((long long)heads * (kHeadDim / 8)));
+  const uint4 raw = __ldcs(in + idx);
+  const float4* tp = reinterpret_cast<const float4*>(table + (long long)r * kPairs + chunk * 4);
+  const float4 t01 = __ldg(tp);
+  const float4 t23 = __ldg(tp + 1);
+  const float2 e0 = unpack_bf16(raw.x), e1 = unpack_bf16(raw.y), e2 = unpack_bf16(raw.z), e3 = unpack_bf16(raw.w);
+  uint4 o;
+  o.x = pack_bf16(e0.x * t01.x - e0.y * t01.y, e0.x * t01.y + e0.y * t01.x);
+  o.y = pack_bf16(e1.x * t01.z - e1.y * t01.w, e1.x * t01.w + e1.y * t01.z);
+  o.z = pack_bf16(e2.x * t23.x - e2.y * t23.y, e2.x * t23.y + e2.y * t23.x);
+  o.w = pack_bf16(e3.x * t23.z - e3.y * t23.w, e3.x * t23.w + e3.y * t23.z);
+  __stcs(out + idx, o);
+}
+
+int launch_rope_apply(const __nv_bfloat16* in, __nv_bfloat16* out, const float2* table, int rows, int heads,
+                      cudaStream_t s) {
+  const long long total = (long long)rows * heads * (kHeadDim / 8);
+  if (total <= 0) return 0;
+  const int blocks = (int)((total + 255) / 256);
+  rope_apply_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out),
+                                           table, rows, heads);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ positions
+// (t, h, w, l) of each token of [text | image | refs]: text i at l = i; image
+// token (r, c) of the token grid at (h, w) = (r, c); reference k at the same
+// grid coordinates with l = -(k + 1) (blog RoPE table; Chinese summary page).
+
+struct RefDims {
+  int n;
+  int h[10];
+  int w[10];
+};
+
+__global__ void positions_kernel(float* __restrict__ pos, int n_txt, int img_h, int img_w, RefDims refs,
+                                 int total) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= total) return;
+  float t = 0.f, hh = 0.f, ww = 0.f, l = 0.f;
+  const int n_img = img_h * img_w;
+  if (r < n_txt) {
+    l = static_cast<float>(r);
+  } else if (r < n_txt + n_img) {
+    const int i = r - n_txt;
+    hh = static_cast<float>(i / img_w);
+    ww = static_cast<float>(i % img_w);
+  } else {
+    int i = r - n_txt - n_img;
+    for (int k = 0; k < refs.n; ++k) {
+      const int cnt = refs.h[k] * refs.w[k];
+      if (i < cnt) {
+        hh = static_cast<float>(i / refs.w[k]);
+        ww = static_cast<float>(i % refs.w[k]);
+        l = static_cast<float>(-(k + 1));
+        break;
+      }
+      i -= cnt;
+    }
+  }
+  reinterpret_cast<float4*>(pos)[r] = make_float4(t, hh, ww, l);
+}
+
+int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, const int* ref_h, const int* ref_w,
+                     cudaStream_t s) {
+  RefDims rd{};
+  rd.n = n_refs;
+  int total = n_txt + img_h * img_w;
+  for (int k = 0; k < n_refs && k < 10; ++k) {
+    rd.h[k] = ref_h[k];
+    rd.w[k] = ref_w[k];
+    total += ref_h[k] * ref_w[k];
+  }
+  if (total <= 0) return 0;
+  positions_kernel<<<(total + 255) / 256, 256, 0, s>>>(pos, n_txt, img_h, img_w, rd, total);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ Euler + CFG
+// x <- x + (sigma_next - sigma) * v, v = v_u + g (v_c - v_u) when v_u is given
+// (guide "How to Run FLUX 3 Image Klein Locally", "The denoise loop" and
+// "Why dropping CFG halves the compute"); optional x0 = x - sigma * v.
+
+__global__ void euler_kernel(float4* __restrict__ x, const float4* __restrict__ vc, const float4* __restrict__ vu,
+                             long long n4, float dsigma, float g, float4* __restrict__ x0, float sigma) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 v = __ldcs(vc + i);
+  if (vu) {
+    const float4 u = __ldcs(vu + i);
+    v.x = fmaf(g, v.x - u.x, u.x);
+    v.y = fmaf(g, v.y - u.y, u.y);
+    v.z = fmaf(g, v.z - u.z, u.z);
+    v.w = fmaf(g, v.w - u.w, u.w);
+  }
+  const float4 xv = x[i];
+  if (x0) x0[i] = make_float4(fmaf(-sigma, v.x, xv.x), fmaf(-sigma, v.y, xv.y), fmaf(-sigma, v.z, xv.z),
+                              fmaf(-sigma, v.w, xv.w));
+  x[i] = make_float4(fmaf(dsigma, v.x, xv.x), fmaf(dsigma, v.y, xv.y), fmaf(dsigma, v.z, xv.z),
+                     fmaf(dsigma, v.w, xv.w));
+}
+
+int launch_euler(float* x, const float* vc, const float* vu, long long n, float dsigma, float g, float* x0,
+                 float sigma, cudaStream_t s) {
+  if (n <= 0) return 0;
+  const long long n4 = n / 4;
+  const int blocks = (int)((n4 + 255) / 256);
+  euler_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(vc),
+                                      reinterpret_cast<const float4*>(vu), n4, dsigma, g,
+                                      reinterpret_cast<float4*>(x0), sigma);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+__global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, long long n4) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = in[i];
+  out[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+}
+
+int launch_to_bf16(const float* in, __nv_bfloat16* out, long long n, cudaStream_t s) {
+  if (n <= 0) return 0;
+  const long long n4 = n / 4;
+  to_bf16_kernel<<<(int)((n4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(in),
+                                                         reinterpret_cast<uint2*>(out), n4);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ GEMV
+// y[v][n] = sum_k W[n][k] * f(x[v][k]) (+ add[n]), f = SiLU or identity,
+// W bf16 [n_out][k] streamed once for up to 4 vectors. One warp per row.
+
+constexpr int kMaxVec = 4;
+
+__global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restrict__ w, int n_out, int k,
+                                                   const float* __restrict__ x, int n_vec, long long x_stride,
+                                                   float* __restrict__ y, long long y_stride, int act_silu,
+                                                   const float* __restrict__ add) {
+  extern __shared__ float xs[];  // [n_vec][k]
+  for (int i = threadIdx.x; i < n_vec * k; i += blockDim.x) {
+    const int vv = i / k;
+    const float e = x[vv * x_stride + (i % k)];
+    xs[i] = act_silu ? silu(e) : e;
+  }
+  __syncthreads();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_out) return;
+  const uint4* wr = reinterpret_cast<const uint4*>(w + (long long)row * k);
+  float acc[kMaxVec] = {0.f, 0.f, 0.f, 0.f};
+  for (int c = lane; c < k / 8; c += 32) {
+    const uint4 raw = __ldcs(wr + c);
+    const float2 w0 = unpack_bf16(raw.x), w1 = unpack_bf16(raw.y), w2 = unpack_bf16(raw.z), w3 = unpack_bf16(raw.w);
+#pragma unroll
+    for (int vv = 0; vv < kMaxVec; ++vv) {
+      if (vv >= n_vec) break;
+      const float* xv = xs + vv * k + 8 * c;
+      float a = acc[vv];
+      a = fmaf(w0.x, xv[0], a); a = fmaf(w0.y, xv[1], a); a = fmaf(w1.x, xv[2], a); a = fmaf(w1.y, xv[3], a);
+      a = fmaf(w2.x, xv[4], a); a = fmaf(w2.y, xv[5], a); a = fmaf(w3.x, xv[6], a); a = fmaf(w3.y, xv[7], a);
+      acc[vv] = a;
+    }
+  }
+#pragma unroll
+  for (int vv = 0; vv < kMaxVec; ++vv) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc[vv] += __shfl_xor_sync(0xffffffffu, acc[vv], o);
+  }
+  if (lane == 0) {
+    const float ad = add ? add[row] : 0.f;
+    for (int vv = 0; vv < n_vec; ++vv) y[vv * y_stride + row] = acc[vv] + ad;
+  }
+}
+
+int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_vec, long long x_stride, float* y,
+                long long y_stride, int act_silu, const float* add, cudaStream_t s) {
+  if (n_vec < 1 || n_vec > kMaxVec || (k % 8) != 0) return -2;
+  const size_t smem = sizeof(float) * n_vec * k;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxVec * kDim * 4) !=
+        cudaSuccess)
+      return -1;
+    configured = true;
+  }
+  gemv_kernel<<<(n_out + 7) / 8, 256, smem, s>>>(w, n_out, k, x, n_vec, x_stride, y, y_stride, act_silu, add);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ time embedding + modulation
+// READING of the pages: the sinusoid of 1000 * sigma is [cos(t f_j), sin(t f_j)]
+// with f_j = 10000^(-j/128); the embedder is Linear -> SiLU -> Linear without
+// biases (guide "What step distillation removed"); the distilled target-level
+// embedder's output is added to every mode's embedding; modulation is
+// W * SiLU(e) split into (shift, scale, gate).
+
+__global__ void sinusoid_kernel(float* __restrict__ out, float t0, float t1, float t2) {
+  const int i = threadIdx.x;  // 0..127
+  const int v = blockIdx.x;   // 0..2
+  const double t = 1000.0 * static_cast<double>(v == 0 ? t0 : (v == 1 ? t1 : t2));
+  const double f = pow(10000.0, -static_cast<double>(i) / 128.0);
+  double sn, cs;
+  sincos(t * f, &sn, &cs);
+  out[v * 256 + i] = static_cast<float>(cs);
+  out[v * 256 + 128 + i] = static_cast<float>(sn);
+}
+
+int launch_time_mod(const TimeModArgs& a, cudaStream_t s) {
+  // scratch layout (floats): sin[3][256] | h1[2][3072] | e[2][3072] | tg1[3072] | tg[3072]
+  float* sin_v = a.scratch;
+  float* h1 = sin_v + 3 * 256;
+  float* e = h1 + 2 * kDim;
+  float* tg1 = e + 2 * kDim;
+  float* tg = tg1 + kDim;
+  sinusoid_kernel<<<3, 128, 0, s>>>(sin_v, a.sigma, 0.0f, a.sigma_next);
+  note_launch();
+  if (cudaGetLastError() != cudaSuccess) return -1;
+  const float* add = nullptr;
+  if (a.tt_mlp1) {
+    if (launch_gemv(a.tt_mlp1, kDim, 256, sin_v + 2 * 256, 1, 256, tg1, kDim, 0, nullptr, s)) return -1;
+    if (launch_gemv(a.tt_mlp2, kDim, kDim, tg1, 1, kDim, tg, kDim, 1, nullptr, s)) return -1;
+    add = tg;
+  }
+  // e[0] = image (sigma), e[1] = context streams (t = 0)
+  if (launch_gemv(a.t_mlp1, kDim, 256, sin_v, 2, 256, h1, kDim, 0, nullptr, s)) return -1;
+  if (launch_gemv(a.t_mlp2, kDim, kDim, h1, 2, kDim, e, kDim, 1, add, s)) return -1;
+  const float* e_img = e;
+  const float* e_ctx = e + kDim;
+  for (int st = 0; st < 2; ++st) {
+    for (int m = 0; m < 3; ++m) {
+      if (m == 2 && !a.with_ref) continue;
+      const float* ev = (m == 1) ? e_img : e_ctx;
+      float* out = a.mod_out + (st * 3 + m) * 3 * kDim;
+      if (launch_gemv(a.mod[st][m], 3 * kDim, kDim, ev, 1, kDim, out, 3 * kDim, 1, nullptr, s)) return -1;
+    }
+  }
+  return launch_gemv(a.final_mod, 2 * kDim, kDim, e_img, 1, kDim, a.final_out, 2 * kDim, 1, nullptr, s);
+}
+
+// ------------------------------------------------------------------ bounded-wait probe
+// Waits on an mbarrier that nothing arrives on, with the given limit, and
+// records kErrTimeout. Exercises the same try_wait + %globaltimer bound as
+// every pipeline wait, without touching any other kernel.
+
+__global__ void wait_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+      if (mbar_try_wait(&bar, 0)) break;
+      if ((i & 63u) == 0u && globaltimer() - t0 > limit_ns) {
+        record_error(kErrTimeout, 0x900);
+        break;
+      }
+    }
+  }
+}
+
+int launch_wait_probe(unsigned long long limit_ns, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace klein

@@ -8,6 +8,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def ensure_built():
+    """Compile libklein.so if it is missing or older than its sources."""
+    import importlib.util
+    path = os.path.join(ROOT, "latent_flow_matching_joint_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("klein_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long CPU oracle run")

@@ -1,0 +1,112 @@
+"""CPU tests of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-only functions (schedule, padding, sequence counts,
+argument checks) agree with the oracle. No device work is issued."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kb():
+    from conftest import ensure_built
+    ensure_built()
+    import latent_flow_matching_joint_b200 as kb
+    return kb
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "klein.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(klein_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(kb):
+    declared = header_functions()
+    assert len(declared) >= 20
+    for name in declared:
+        assert hasattr(kb.lib, name), name
+    # the binding wraps exactly the declared C functions
+    assert sorted(kb.EXPORTED) == declared
+
+
+def test_schedule_matches_oracle(kb):
+    for steps in (1, 4, 16, 50):
+        got = np.array(kb.klein_sigma_schedule(steps))
+        np.testing.assert_allclose(got, o.sigma_schedule(steps), rtol=0, atol=6e-8)
+    assert kb.klein_sigma_schedule(16)[-1] == 0.0
+
+
+def test_pad_text_len_matches_oracle(kb):
+    for n in (0, 1, 79, 80, 81, 160, 512, 1000):
+        assert kb.klein_pad_text_len(n) == o.pad_text_len(n)
+    assert kb.klein_pad_text_len(-1) == -1
+
+
+def test_seq_tokens(kb):
+    s = kb.make_seq(1, 512, 64, 64)
+    assert kb.klein_seq_tokens(s) == (4096, 0, 4608)
+    s = kb.make_seq(1, 512, 64, 64, refs=[(64, 64)])
+    assert kb.klein_seq_tokens(s) == (4096, 4096, 8704)
+    s = kb.make_seq(2, 560, 128, 128)
+    assert kb.klein_seq_tokens(s) == (16384, 0, 16944)
+    assert kb.klein_seq_tokens(kb.make_seq(1, 80, 8, 8)) == (64, 0, 144)
+
+
+def test_seq_errors(kb):
+    for bad in (kb.make_seq(0, 10, 2, 2), kb.make_seq(1, 0, 2, 2), kb.make_seq(1, 5, 0, 2)):
+        with pytest.raises(kb.KleinError) as e:
+            kb.klein_seq_tokens(bad)
+        assert e.value.name == "KLEIN_ERR_SHAPE"
+    s = kb.make_seq(1, 5, 2, 2)
+    s.n_refs = 11
+    with pytest.raises(kb.KleinError):
+        kb.klein_seq_tokens(s)
+
+
+def test_workspace_sizes_grow(kb):
+    a = kb.klein_block_workspace_size(1, 144)
+    b = kb.klein_block_workspace_size(1, 4608)
+    c = kb.klein_block_workspace_size(2, 4608)
+    assert 0 < a < b < c
+    assert kb.klein_block_workspace_size(0, 10) == 0
+    s1 = kb.klein_stack_workspace_size(kb.make_seq(1, 512, 64, 64))
+    assert s1 > kb.klein_block_workspace_size(1, 4608)
+
+
+def test_argument_errors_before_any_launch(kb):
+    bw = kb.KleinBlockWeights(None, None, None, None)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), None, 1, 10, 0, 10, 5, 5, None, None, None, 0, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
+    assert b"incomplete" in kb.lib.klein_last_error()
+    # misaligned weights
+    bw = kb.KleinBlockWeights(16, 18, 32, 48)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), None, 1, 10, 0, 10, 5, 5, None, None, None, 0, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_ALIGN"
+    # bad range
+    bw = kb.KleinBlockWeights(16, 32, 48, 64)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 5, 10, 5, 5, 256, 256, 256, 1 << 30, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    # workspace too small
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1024, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_WORKSPACE"
+    rc = kb.lib.klein_op_gemm(256, 256, 256, 10, 100, 64, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    rc = kb.lib.klein_op_euler(256, 256, None, 6, ctypes.c_float(0.1), ctypes.c_float(1.0), None,
+                               ctypes.c_float(0.0), None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    assert kb.lib.klein_wait_probe(0, None) == -1
+
+
+def test_model_create_validation(kb):
+    d = kb.KleinModelDesc()
+    d.n_stage1, d.n_joint = 0, 0
+    h = ctypes.c_void_p()
+    rc = kb.lib.klein_model_create(ctypes.byref(h), ctypes.byref(d))
+    assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
