@@ -363,7 +363,7 @@ def run_ours(args):
     jb = None
     if args.workload == "t2i":
         bw = model_t["joint"][0]
-        x = torch.randn(1, 4608, DIM, generator=g, device=dev).to(torch.bfloat16)
+        x = torch.randn(1, 4608, DIM, generator=g, device=dev)
         pos = torch.empty(4608, 4, device=dev)
         kb.klein_positions(kb.make_seq(1, 512, 64, 64), pos)
         mod = 0.5 * torch.randn(3, 3, DIM, generator=g, device=dev)

@@ -163,7 +163,8 @@ size_t klein_block_workspace_size(int batch, int rows);
  * `rows` rows only, no mask; x += gate * (attention out-projection + MLP).
  * A joint block passes row0 = 0, rows = n_total; a stage-1 block passes one
  * stream's row range (each stream attends only to itself).
- *   x        device bf16 [batch][n_total][3072], updated in place
+ *   x        device float [batch][n_total][3072] (the residual stream is
+ *            kept in fp32), updated in place
  *   pos      device float [n_total][4] (klein_positions)
  *   mod      device float [3 modes][3 (shift, scale, gate)][3072]
  *   ws       device workspace, >= klein_block_workspace_size(batch, rows)
@@ -237,7 +238,7 @@ int klein_denoise(const klein_model* m, float* latents, const void* text, const 
 /* h = modulated LayerNorm of rows [row0, row0 + rows) of x (mode by global
  * row as in klein_block_forward). mod: [3][>=2][3072] with per-mode stride
  * mod_stride floats; single_mode != 0 applies mod[0] to every row.
- * x: bf16 [batch][n_total][3072]; h: bf16 [batch][rows][3072]. */
+ * x: float [batch][n_total][3072]; h: bf16 [batch][rows][3072]. */
 int klein_op_modln(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
                    const float* mod, long long mod_stride, int single_mode, void* h, void* stream);
 

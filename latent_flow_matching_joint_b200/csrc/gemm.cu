@@ -150,25 +150,23 @@ __device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int
   const int grow = g.x_row0 + r;
   const int mode = mode_of_row(grow, g.n_txt, g.n_img);
   const float* gate = g.mod + (long long)mode * 3 * kDim + 2 * kDim + n_idx * BN;
-  __nv_bfloat16* xr = g.x + ((long long)b * g.x_bstride + grow) * kDim + n_idx * BN;
+  float* xr = g.x + ((long long)b * g.x_bstride + grow) * kDim + n_idx * BN;
   float v[32];
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     tmem_ld32(taddr + 32 * c, v);
     if (!valid) continue;
-    __nv_bfloat16* p = xr + 32 * c;
-    const float* gt = gate + 32 * c;
+    float4* p = reinterpret_cast<float4*>(xr + 32 * c);
+    const float4* gt = reinterpret_cast<const float4*>(gate + 32 * c);
 #pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-      uint4 raw = *reinterpret_cast<const uint4*>(p + i);
-      float2 a0 = unpack_bf16(raw.x), a1 = unpack_bf16(raw.y), a2 = unpack_bf16(raw.z), a3 = unpack_bf16(raw.w);
-      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gt + i));
-      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gt + i + 4));
-      raw.x = pack_bf16(fmaf(g0.x, v[i + 0], a0.x), fmaf(g0.y, v[i + 1], a0.y));
-      raw.y = pack_bf16(fmaf(g0.z, v[i + 2], a1.x), fmaf(g0.w, v[i + 3], a1.y));
-      raw.z = pack_bf16(fmaf(g1.x, v[i + 4], a2.x), fmaf(g1.y, v[i + 5], a2.y));
-      raw.w = pack_bf16(fmaf(g1.z, v[i + 6], a3.x), fmaf(g1.w, v[i + 7], a3.y));
-      *reinterpret_cast<uint4*>(p + i) = raw;
+    for (int i = 0; i < 8; ++i) {
+      float4 xv = p[i];
+      const float4 gv = __ldg(gt + i);
+      xv.x = fmaf(gv.x, v[4 * i + 0], xv.x);
+      xv.y = fmaf(gv.y, v[4 * i + 1], xv.y);
+      xv.z = fmaf(gv.z, v[4 * i + 2], xv.z);
+      xv.w = fmaf(gv.w, v[4 * i + 3], xv.w);
+      p[i] = xv;
     }
   }
 }

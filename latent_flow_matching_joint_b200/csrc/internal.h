@@ -51,7 +51,7 @@ struct GemmArgs {
   const float2* rope;  // [rows][64] (cos, sin)
   int rows_pad;
   // kEpiResid
-  __nv_bfloat16* x;   // [batch][x_bstride rows][3072]
+  float* x;           // residual stream, fp32 [batch][x_bstride rows][3072]
   long long x_bstride;
   int x_row0;
   const float* mod;   // [3 modes][3][3072] (shift, scale, gate)
@@ -76,7 +76,7 @@ int launch_attention(const CUtensorMap& map_q, const CUtensorMap& map_k, const C
 
 // ------------------------------------------------------------------ memory-bound kernels
 
-int launch_modln(const __nv_bfloat16* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
+int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
                  int n_txt, int n_img, const float* mod, long long mod_mode_stride, int single_mode,
                  cudaStream_t stream);
 int launch_rope_table(const float* pos, float2* table, int rows, float theta, cudaStream_t stream);
@@ -87,8 +87,8 @@ int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, co
 int launch_euler(float* x, const float* v_cond, const float* v_uncond, long long n, float dsigma, float g,
                  float* x0_out, float sigma, cudaStream_t stream);
 int launch_to_bf16(const float* in, __nv_bfloat16* out, long long n, cudaStream_t stream);
-int launch_copy_rows(const __nv_bfloat16* src, long long src_bstride, __nv_bfloat16* dst, long long dst_bstride,
-                     int dst_row0, int batch, int rows, int src_batches, cudaStream_t stream);
+int launch_rows_to_f32(const __nv_bfloat16* src, long long src_bstride, float* dst, long long dst_bstride,
+                       int dst_row0, int batch, int rows, cudaStream_t stream);
 
 // Timestep embedding + modulation (a2).
 struct TimeModArgs {

@@ -13,9 +13,11 @@ namespace klein {
 // with m the row's stream (Diffusers release blog for FLUX.3 Klein, "Speed,
 // architecture, and how the tokens move": no learned affine; text and
 // reference rows take the t = 0 modulation, image rows the current t).
-// One warp per row; 12 x 16-byte loads per lane; fp32 statistics.
+// The residual stream x is fp32; h is the bf16 A operand of the
+// in-projection. One warp per row: 24 x 16-byte loads per lane, fp32
+// statistics (two passes over registers), 8-byte bf16 stores.
 
-__global__ void __launch_bounds__(256, 2) modln_kernel(const __nv_bfloat16* __restrict__ x, long long x_bstride,
+__global__ void __launch_bounds__(256, 2) modln_kernel(const float* __restrict__ x, long long x_bstride,
                                                     int x_row0, __nv_bfloat16* __restrict__ h, int batch,
                                                     int rows, int n_txt, int n_img,
                                                     const float* __restrict__ mod, long long mod_stride,
@@ -26,67 +28,78 @@ __global__ void __launch_bounds__(256, 2) modln_kernel(const __nv_bfloat16* __re
   const int b = warp / rows;
   const int i = warp % rows;
   const int grow = x_row0 + i;
-  const uint4* src = reinterpret_cast<const uint4*>(x + ((long long)b * x_bstride + grow) * kDim);
-  uint4* dst = reinterpret_cast<uint4*>(h + ((long long)b * rows + i) * kDim);
-  constexpr int kVec = kDim / 8 / 32;  // 12 uint4 per lane, kept packed
-  uint4 raw[kVec];
+  const float4* src = reinterpret_cast<const float4*>(x + ((long long)b * x_bstride + grow) * kDim);
+  uint2* dst = reinterpret_cast<uint2*>(h + ((long long)b * rows + i) * kDim);
+  constexpr int kVec = kDim / 4 / 32;  // 24 float4 per lane
+  float4 v[kVec];
 #pragma unroll
-  for (int t = 0; t < kVec; ++t) raw[t] = __ldcs(src + lane + 32 * t);
+  for (int t = 0; t < kVec; ++t) v[t] = __ldg(src + lane + 32 * t);
   float sum = 0.f;
 #pragma unroll
-  for (int t = 0; t < kVec; ++t) {
-    const uint32_t w4[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 e = unpack_bf16(w4[q]);
-      sum += e.x + e.y;
-    }
-  }
+  for (int t = 0; t < kVec; ++t) sum += (v[t].x + v[t].y) + (v[t].z + v[t].w);
 #pragma unroll
   for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float mean = sum * (1.0f / kDim);
   float sq = 0.f;
 #pragma unroll
   for (int t = 0; t < kVec; ++t) {
-    const uint32_t w4[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 e = unpack_bf16(w4[q]);
-      const float d0 = e.x - mean, d1 = e.y - mean;
-      sq = fmaf(d0, d0, fmaf(d1, d1, sq));
-    }
+    const float a = v[t].x - mean, bb = v[t].y - mean, c = v[t].z - mean, d = v[t].w - mean;
+    sq = fmaf(a, a, fmaf(bb, bb, fmaf(c, c, fmaf(d, d, sq))));
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   const float rstd = rsqrtf(sq * (1.0f / kDim) + 1e-6f);
   const int m = single_mode ? 0 : mode_of_row(grow, n_txt, n_img);
-  const float* shift = mod + m * mod_stride;
-  const float* scale = shift + kDim;
+  const float4* shift = reinterpret_cast<const float4*>(mod + m * mod_stride);
+  const float4* scale = reinterpret_cast<const float4*>(mod + m * mod_stride + kDim);
 #pragma unroll
   for (int t = 0; t < kVec; ++t) {
-    const int col = 8 * (lane + 32 * t);
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(scale + col));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(scale + col + 4));
-    const float4 h0 = __ldg(reinterpret_cast<const float4*>(shift + col));
-    const float4 h1 = __ldg(reinterpret_cast<const float4*>(shift + col + 4));
-    const float2 e0 = unpack_bf16(raw[t].x), e1 = unpack_bf16(raw[t].y);
-    const float2 e2 = unpack_bf16(raw[t].z), e3 = unpack_bf16(raw[t].w);
-    uint4 o;
-    o.x = pack_bf16(fmaf((e0.x - mean) * rstd, 1.f + s0.x, h0.x), fmaf((e0.y - mean) * rstd, 1.f + s0.y, h0.y));
-    o.y = pack_bf16(fmaf((e1.x - mean) * rstd, 1.f + s0.z, h0.z), fmaf((e1.y - mean) * rstd, 1.f + s0.w, h0.w));
-    o.z = pack_bf16(fmaf((e2.x - mean) * rstd, 1.f + s1.x, h1.x), fmaf((e2.y - mean) * rstd, 1.f + s1.y, h1.y));
-    o.w = pack_bf16(fmaf((e3.x - mean) * rstd, 1.f + s1.z, h1.z), fmaf((e3.y - mean) * rstd, 1.f + s1.w, h1.w));
-    dst[lane + 32 * t] = o;
+    const int c4 = lane + 32 * t;
+    const float4 sc = __ldg(scale + c4);
+    const float4 sh = __ldg(shift + c4);
+    const float4 e = v[t];
+    dst[c4] = make_uint2(pack_bf16(fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x), fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y)),
+                         pack_bf16(fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z), fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w)));
   }
 }
 
-int launch_modln(const __nv_bfloat16* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
+int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
                  int n_txt, int n_img, const float* mod, long long mod_stride, int single_mode, cudaStream_t s) {
   const long long warps = (long long)batch * rows;
   if (warps <= 0) return 0;
   const int blocks = (int)((warps + 7) / 8);
   modln_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, h, batch, rows, n_txt, n_img, mod, mod_stride,
                                       single_mode);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// bf16 rows -> fp32 rows of the residual stream: src [batch][rows][3072]
+// (batch stride src_bstride rows) into dst rows [dst_row0, dst_row0 + rows)
+// of each batch item (batch stride dst_bstride rows).
+__global__ void rows_to_f32_kernel(const uint4* __restrict__ src, long long src_bstride, float4* __restrict__ dst,
+                                   long long dst_bstride, int dst_row0, int rows, long long total) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  constexpr int kPerRow = kDim / 8;
+  const long long row = idx / kPerRow;
+  const int c = static_cast<int>(idx % kPerRow);
+  const long long b = row / rows;
+  const long long r = row % rows;
+  const uint4 raw = __ldg(src + (b * src_bstride + r) * kPerRow + c);
+  const float2 a = unpack_bf16(raw.x), bb = unpack_bf16(raw.y), cc = unpack_bf16(raw.z), d = unpack_bf16(raw.w);
+  float4* o = dst + ((b * dst_bstride + dst_row0 + r) * kPerRow + c) * 2;
+  o[0] = make_float4(a.x, a.y, bb.x, bb.y);
+  o[1] = make_float4(cc.x, cc.y, d.x, d.y);
+}
+
+int launch_rows_to_f32(const __nv_bfloat16* src, long long src_bstride, float* dst, long long dst_bstride,
+                       int dst_row0, int batch, int rows, cudaStream_t s) {
+  const long long total = (long long)batch * rows * (kDim / 8);
+  if (total <= 0) return 0;
+  rows_to_f32_kernel<<<(int)((total + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(src), src_bstride,
+                                                                  reinterpret_cast<float4*>(dst), dst_bstride,
+                                                                  dst_row0, rows, total);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -155,7 +155,7 @@ static BlockWs carve_block(void* base, int batch, int rows) {
 
 // One block over rows [row0, row0+rows) of x. `rope` holds the view's table
 // (row 0 = global row row0). Workspace `w` is carved for (batch, >= rows).
-static int block_impl(const klein_block_weights* wt, __nv_bfloat16* x, int batch, int n_total, int row0, int rows,
+static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_total, int row0, int rows,
                       int n_txt, int n_img, const float2* rope, const float* mod, const BlockWs& w,
                       cudaStream_t s) {
   const int rp = round_up(rows, 128);
@@ -248,7 +248,7 @@ static int check_seq(const klein_seq* q, int* n_img, int* n_ref, int* n_total) {
 // ------------------------------------------------------------------ stack
 
 struct StackWs {
-  __nv_bfloat16* x;
+  float* x;           // residual stream [batch][n_total][3072]
   float* pos;
   float2* rope;
   float* mod;        // [2][3][3][3072]
@@ -268,7 +268,7 @@ static StackWs carve_stack(void* base, int batch, int n_total, int n_img, int n_
     off += align256(n);
     return p;
   };
-  w.x = reinterpret_cast<__nv_bfloat16*>(take((size_t)batch * n_total * kDim * 2));
+  w.x = reinterpret_cast<float*>(take((size_t)batch * n_total * kDim * sizeof(float)));
   w.pos = reinterpret_cast<float*>(take((size_t)n_total * 4 * sizeof(float)));
   w.rope = reinterpret_cast<float2*>(take((size_t)n_total * kPairs * sizeof(float2)));
   w.mod = reinterpret_cast<float*>(take((size_t)2 * 3 * 3 * kDim * sizeof(float)));
@@ -443,7 +443,7 @@ int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_
   if (ws_bytes < bw.bytes) return fail(KLEIN_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, bw.bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_rope_table(pos + (size_t)row0 * 4, bw.rope, rows, 10000.f, s)) return cuda_fail("rope table");
-  return block_impl(w, static_cast<__nv_bfloat16*>(x), batch, n_total, row0, rows, n_txt, n_img, bw.rope, mod, bw,
+  return block_impl(w, static_cast<float*>(x), batch, n_total, row0, rows, n_txt, n_img, bw.rope, mod, bw,
                     s);
 }
 
@@ -528,12 +528,8 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
   prof_end(pi, s);
   // a3: assemble [text | image | reference] rows of x
   pi = prof_begin(kProfOther, s);
-  for (int b = 0; b < B; ++b) {
-    if (cudaMemcpyAsync(w.x + (size_t)b * n_total * kDim, static_cast<const __nv_bfloat16*>(text) +
-                                                              (size_t)b * n_txt * kDim,
-                        (size_t)n_txt * kDim * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return cuda_fail("text copy");
-  }
+  if (launch_rows_to_f32(static_cast<const __nv_bfloat16*>(text), n_txt, w.x, n_total, 0, B, n_txt, s))
+    return cuda_fail("text rows");
   prof_end(pi, s);
   auto project = [&](const float* lat, int rows, const void* wproj, int row0) -> int {
     const int pc = prof_begin(kProfProj, s);
@@ -555,7 +551,7 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
     g.out_row0 = row0;
     g.replicate = B;
     const int pj = prof_begin(kProfProj, s);
-    if (launch_gemm(256, kEpiBF16, ma, mb, g, s)) return cuda_fail("input projection launch");
+    if (launch_gemm(256, kEpiF32, ma, mb, g, s)) return cuda_fail("input projection launch");
     prof_end(pj, s);
     return KLEIN_OK;
   };
@@ -678,7 +674,7 @@ int klein_op_modln(const void* x, int batch, int n_total, int row0, int rows, in
   if (!aligned16(x) || !aligned16(mod) || !aligned16(h) || (mod_stride % 4) != 0)
     return fail(KLEIN_ERR_ALIGN, "pointers must be 16-byte aligned, mod_stride a multiple of 4");
   if (batch < 1 || rows < 1 || row0 < 0 || row0 + rows > n_total) return fail(KLEIN_ERR_SHAPE, "bad row range");
-  if (launch_modln(static_cast<const __nv_bfloat16*>(x), n_total, row0, static_cast<__nv_bfloat16*>(h), batch, rows,
+  if (launch_modln(static_cast<const float*>(x), n_total, row0, static_cast<__nv_bfloat16*>(h), batch, rows,
                    n_txt, n_img, mod, mod_stride, single_mode, static_cast<cudaStream_t>(stream)))
     return cuda_fail("modln launch");
   return KLEIN_OK;

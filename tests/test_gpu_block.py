@@ -33,7 +33,7 @@ def weights():
 
 def run_block(kb, wd, x, seq, mod, row0, rows, n_txt, n_img):
     batch, n_total = x.shape[0], x.shape[1]
-    xd = to_bf16(x)
+    xd = to_f32(x)
     pos = torch.empty((n_total, 4), dtype=torch.float32, device="cuda")
     kb.klein_positions(seq, pos)
     ws = workspace(kb.klein_block_workspace_size(batch, rows))
