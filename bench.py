@@ -180,7 +180,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = args.workload
+    wl = args.workload if args.workload in WORKLOADS else "t2i"
     for _ in range(args.warmup):
         oracle_block_sample(80, (8, 8))
     times = [oracle_block_sample() for _ in range(args.steps)]
@@ -236,10 +236,50 @@ def random_model(dev, distilled, with_ref, seed=0):
     return t
 
 
+def run_block_only(args):
+    """Times klein_block_forward alone: one joint block over 512 text + 64x64
+    image tokens (the 1024x1024 configuration), batch 1. A small case for
+    kernel profiles (about 1.3 GB of device memory)."""
+    import torch
+    import latent_flow_matching_joint_b200 as kb
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    bw = random_block(g, dev)
+    x = torch.randn(1, 4608, DIM, generator=g, device=dev)
+    pos = torch.empty(4608, 4, device=dev)
+    kb.klein_positions(kb.make_seq(1, 512, 64, 64), pos)
+    mod = 0.5 * torch.randn(3, 3, DIM, generator=g, device=dev)
+    ws = torch.empty(kb.klein_block_workspace_size(1, 4608), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        kb.klein_block_forward(bw, x, 512, 4096, pos, mod, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s = torch.cuda.current_stream()
+    e0.record(s)
+    for _ in range(args.steps):
+        kb.klein_block_forward(bw, x, 512, 4096, pos, mod, ws)
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    flops = 4608 * block_gemm_flops_per_token() + attn_flops(4608)
+    peaks = load_peaks()
+    rc, _, msg = kb.klein_device_status()
+    if rc != 0:
+        raise RuntimeError(msg)
+    print(json.dumps({"metric": "joint-block TFLOP/s at 512+4096 tokens", "value": flops / (ms / 1e3) / 1e12,
+                      "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16"], "dtype": "bf16",
+                      "config": {"workload": "one joint block, 512 text + 64x64 image tokens, batch 1"}}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
+    if args.workload == "block":
+        return run_block_only(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -420,7 +460,7 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=tuple(WORKLOADS), default="t2i")
+    ap.add_argument("--workload", choices=tuple(WORKLOADS) + ("block",), default="t2i")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

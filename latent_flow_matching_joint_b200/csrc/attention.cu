@@ -5,17 +5,23 @@
 // padding included; in stage 1 each stream attends to itself, which the
 // caller expresses as a view over that stream's rows).
 //
-// One CTA = one 128-row query tile of one head. Roles (192 threads):
-//   warp 0      TMA: Q once, then K and V^T tiles of 128 keys, 2 stages
-//   warp 1      TMEM allocator and MMA issuer: S = Q K^T into one of two
-//               TMEM score buffers (so S_{j+1} overlaps the softmax of S_j),
-//               then O += P V into the TMEM output accumulator
-//   warps 2..5  softmax: one query row per thread, online max / sum in the
-//               exp2 domain, P written to shared memory as bf16 in the
-//               128-byte-swizzled K-major layout the tensor core reads, the
-//               TMEM output row rescaled when the running max grows; final
-//               normalisation and the bf16 store into the out-projection's
-//               A operand.
+// One CTA = two 128-row query tiles (a, b) of one head, sharing every K/V
+// tile. Roles (320 threads):
+//   warp 0      TMA: both Q tiles once, then K and V^T tiles of 128 keys
+//               through a 2-stage ring
+//   warp 1      TMEM allocator and MMA issuer. Per key tile j, for each query
+//               tile t in turn: O_t += P_t V_j (P_t read from tensor memory),
+//               then S_t = Q_t K_{j+1}^T. While one tile's softmax runs, the
+//               tensor core works on the other tile.
+//   warps 2..5  softmax of tile a, warps 6..9 softmax of tile b: one query
+//               row per thread, scores read from TMEM, running max / sum in the
+//               exp2 domain, P written back over the scores in TMEM as bf16.
+//               The running max is only moved (and the TMEM output rescaled)
+//               when a row's max grows by more than 2^8, so rescales are rare;
+//               the bound keeps P <= 256. Final 1/l normalisation and bf16
+//               store into the out-projection's A operand.
+// Tensor memory (512 columns): tile t owns S_t (128 fp32 columns, P_t in its
+// first 64 as packed bf16) and O_t (128 fp32 columns).
 // Keys past the end of the view are zero-filled by TMA and masked to -inf.
 #include <math.h>
 
@@ -26,38 +32,36 @@ namespace klein {
 
 namespace {
 constexpr int kTileBytes = 128 * 128 * 2;  // a 128 x 128 bf16 tile = 2 swizzle chunks of 16 KB
-constexpr int kOffQ = 0;
-constexpr int kOffK = kTileBytes;              // 2 stages
-constexpr int kOffV = 3 * kTileBytes;          // 2 stages
-constexpr int kOffP = 5 * kTileBytes;
+constexpr int kOffQ = 0;                   // 2 query tiles
+constexpr int kOffK = 2 * kTileBytes;      // 2 stages
+constexpr int kOffV = 4 * kTileBytes;      // 2 stages
 constexpr int kOffBar = 6 * kTileBytes;
 constexpr int kSmem = kOffBar + 256 + 1024;
-constexpr uint32_t kTmemCols = 512;            // S0 | S1 | O | unused
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only when the max grows by > 2^8
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_vt, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* v_full = bars + 3;   // [2]
-  uint64_t* kv_empty = bars + 5; // [2]
-  uint64_t* s_full = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2 tiles]: scores ready (phase j), final output ready (phase nkv)
+  uint64_t* p_full = bars + 9;    // [2 tiles]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q_tile = blockIdx.x;
   const int head = blockIdx.y;
   const int b = blockIdx.z;
   const int bh = b * a.heads + head;
-  const int q_row0 = q_tile * 128;
+  const int q_row0 = blockIdx.x * 256;
   const int nkv = (a.rows + 127) / 128;
 
   if (warp == 0 && lane == 0) {
@@ -67,9 +71,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_q);
     tma_prefetch_desc(&map_k);
@@ -87,9 +90,11 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_3d(smem + kOffQ, &map_q, q_full, 0, q_row0, bh);
-      tma_load_3d(smem + kOffQ + kTileBytes / 2, &map_q, q_full, 64, q_row0, bh);
+      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+      for (int t = 0; t < 2; ++t) {
+        tma_load_3d(smem + kOffQ + t * kTileBytes, &map_q, q_full, 0, q_row0 + 128 * t, bh);
+        tma_load_3d(smem + kOffQ + t * kTileBytes + kTileBytes / 2, &map_q, q_full, 64, q_row0 + 128 * t, bh);
+      }
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, 0x201)) break;
@@ -105,113 +110,113 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t q0 = smem_u32(smem + kOffQ);
-      const uint32_t p0 = smem_u32(smem + kOffP);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], (j >> 1) & 1, 0x202)) return false;
-        tc_fence_after();
-        const uint32_t k0 = smem_u32(smem + kOffK + st * kTileBytes);
+      auto issue_s = [&](int t, int j) {
+        const uint32_t q0 = smem_u32(smem + kOffQ + t * kTileBytes);
+        const uint32_t k0 = smem_u32(smem + kOffK + (j & 1) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          umma_bf16(tmem_base + st * 128, sw128_desc(q0 + off), sw128_desc(k0 + off), idesc, kk != 0);
+          umma_bf16(tmem_base + t * 256, sw128_desc(q0 + off), sw128_desc(k0 + off), idesc, kk != 0);
         }
-        umma_commit(&s_full[st]);
-        return true;
+        umma_commit(&s_full[t]);
       };
-      bool ok = mbar_wait(q_full, 0, 0x203);
+      bool ok = mbar_wait(q_full, 0, 0x202) && mbar_wait(&k_full[0], 0, 0x203);
       if (ok) {
         tc_fence_after();
-        ok = issue_s(0);
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv && !issue_s(j + 1)) break;
-        if (!mbar_wait(p_full, j & 1, 0x204)) break;
-        tc_fence_after();
         const int st = j & 1;
-        if (!mbar_wait(&v_full[st], (j >> 1) & 1, 0x205)) break;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(smem + kOffV + st * kTileBytes);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!mbar_wait(&p_full[t], j & 1, 0x204)) { ok = false; break; }
+          if (t == 0 && !mbar_wait(&v_full[st], (j >> 1) & 1, 0x205)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(smem + kOffV + st * kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          umma_bf16(tmem_base + kColO, sw128_desc(p0 + off), sw128_desc(v0 + off), idesc, (j | kk) != 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+            umma_bf16_tmem_a(tmem_base + t * 256 + 128, tmem_base + t * 256 + kk * 8, sw128_desc(v0 + off), idesc,
+                             (j | kk) != 0);
+          }
+          if (t == 1) umma_commit(&kv_empty[st]);
+          if (j + 1 < nkv) {
+            if (t == 0) {
+              if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 0x206)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_s(t, j + 1);
+          } else {
+            umma_commit(&s_full[t]);  // output of tile t final
+          }
         }
-        umma_commit(&kv_empty[st]);
-        umma_commit(o_done);
       }
     }
   } else {
-    const int quarter = warp & 3;
+    const int t = (warp - 2) >> 2;         // query tile of this warpgroup
+    const int quarter = warp & 3;          // TMEM lane quarter of this warp
     const int rloc = quarter * 32 + lane;
-    const int q_row = q_row0 + rloc;
+    const int q_row = q_row0 + 128 * t + rloc;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint8_t* prow = smem + kOffP + rloc * 128;
+    const uint32_t s_col = lane_base + t * 256;
+    const uint32_t o_col = s_col + 128;
     const float sl2 = a.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;
     float s[128];
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (j >> 1) & 1, 0x206)) { ok = false; break; }
+      if (!mbar_wait(&s_full[t], j & 1, 0x207)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + sb * 128 + 32 * c, s + 32 * c);
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_col + 32 * c, s + 32 * c);
       const int lim = a.rows - j * 128;  // valid keys in this tile
-      float mx = -INFINITY;
+      if (lim < 128) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = (i < lim) ? s[i] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : -INFINITY;
       }
-      const float m_new = fmaxf(m_run, mx);
-      float sum = 0.f;
+      float mx = s[0];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = fast_exp2(s[i] - m_new);
-        sum += s[i];
-      }
-      if (j > 0) {
-        if (!mbar_wait(o_done, (j - 1) & 1, 0x207)) { ok = false; break; }
-        tc_fence_after();
-      }
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float m_cand = mx * sl2;
+      // move the running max only if it grows past the threshold
+      const bool grow = m_cand > m_run + kRescaleThreshold;
+      const float m_new = grow ? m_cand : m_run;
       const float alpha = fast_exp2(m_run - m_new);
-      if (j > 0 && __any_sync(0xffffffffu, m_new > m_run)) {
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float p0 = fast_exp2(fmaf(s[i], sl2, -m_new));
+        const float p1 = fast_exp2(fmaf(s[i + 1], sl2, -m_new));
+        sum += p0 + p1;
+        pk[i >> 1] = pack_bf16(p0, p1);
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
         float o[32];
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          tmem_ld32(lane_base + kColO + 32 * c, o);
+          tmem_ld32(o_col + 32 * c, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(lane_base + kColO + 32 * c, o);
+          tmem_st32(o_col + 32 * c, o);
         }
       }
       l_run = l_run * alpha + sum;
       m_run = m_new;
-      // P row -> two 128-byte swizzled chunks (keys 0..63, 64..127)
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int chunk = u >> 3;
-        const int unit = u & 7;
-        uint8_t* dst = prow + chunk * (kTileBytes / 2) + ((unit ^ (rloc & 7)) << 4);
-        const float* p = s + 8 * u;
-        *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                                                    pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-      }
-      fence_proxy_async_smem();
+      tmem_st32(s_col, reinterpret_cast<const float*>(pk));
+      tmem_st32(s_col + 32, reinterpret_cast<const float*>(pk + 32));
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(o_done, (nkv - 1) & 1, 0x208)) {
+    if (ok && mbar_wait(&s_full[t], nkv & 1, 0x208)) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
       __nv_bfloat16* dst = a.out + ((long long)b * a.rows + q_row) * a.out_ld + head * kHeadDim;
       float o[32];
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        tmem_ld32(lane_base + kColO + 32 * c, o);
+        tmem_ld32(o_col + 32 * c, o);
         if (q_row < a.rows) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
@@ -242,8 +247,8 @@ int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     configured = true;
   }
   if (a.rows <= 0 || a.batch <= 0) return 0;
-  dim3 grid((a.rows + 127) / 128, a.heads, a.batch);
-  attn_kernel<<<grid, 192, kSmem, s>>>(mq, mk, mvt, a);
+  dim3 grid((a.rows + 255) / 256, a.heads, a.batch);
+  attn_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mvt, a);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -7,7 +7,9 @@
 //   warps 2..5  epilogue: one accumulator row per thread (TMEM lane quarter
 //               = warp % 4), two accumulator buffers so that the epilogue of
 //               tile i overlaps the main loop of tile i+1.
-// Tiles are visited M-fastest so the CTAs in flight share B tiles in L2.
+// Tiles are visited M-fastest (the CTAs in flight share B tiles in L2 while A
+// stays resident) or N-fastest (B stays resident in L2, each A row block is
+// read from HBM once), whichever operand fits in L2.
 //
 // Epilogues (FLUX.3 Klein block, Diffusers release blog "Speed,
 // architecture, and how the tokens move", and its Chinese translation's
@@ -220,8 +222,8 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const int m_idx = tile % m_tiles;
-        const int n_idx = tile / m_tiles;
+        const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
+        const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
         const int b = m_idx / g.m_tiles_per_b;
         const int row0 = (m_idx % g.m_tiles_per_b) * 128;
         int brow0, brow1;
@@ -279,8 +281,8 @@ __global__ void __launch_bounds__(192, 1)
     const int rloc = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const int m_idx = tile % m_tiles;
-      const int n_idx = tile / m_tiles;
+      const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
+      const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
       const int b = m_idx / g.m_tiles_per_b;
       const int r = (m_idx % g.m_tiles_per_b) * 128 + rloc;
       const int acc = it & 1;

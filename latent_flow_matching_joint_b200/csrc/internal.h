@@ -35,6 +35,7 @@ struct GemmArgs {
   int n_tiles;        // N / BN
   int k_blocks;       // K / 64
   int b_split;        // kEpiQKV: the N-tile where the paired gate|up tiles begin
+  int n_fastest;      // visit tiles N-fastest (B fits in L2, A streamed once) instead of M-fastest
   // kEpiF32 / kEpiBF16: out[(b * out_bstride + out_row0 + r) * out_ld + n]
   void* out;
   long long out_ld;

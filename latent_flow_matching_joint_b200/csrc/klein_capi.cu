@@ -214,6 +214,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   o.m_tiles_per_b = (rows + 127) / 128;
   o.n_tiles = kDim / 256;
   o.k_blocks = kOutK / 64;
+  o.n_fastest = 1;
   o.x = x;
   o.x_bstride = n_total;
   o.x_row0 = row0;
