@@ -173,6 +173,27 @@ int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_
                         int n_txt, int n_img, const float* pos, const float* mod, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* klein_block_forward without a workspace. The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory,
+ * for instance code being recorded into a CUDA graph under global stream
+ * capture (where cudaMalloc is an error), or a plug-in whose device memory
+ * is owned by a host framework's pool that it may not bypass. Same
+ * arguments and results as klein_block_forward, minus ws / ws_bytes.
+ *   - Scratch lives in one fixed array of this library's device memory
+ *     (about 12.1 MiB), held on every GPU that loads the library until the
+ *     process exits. It fits batch * round_up(rows, 128) <= 256; larger
+ *     calls return KLEIN_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero (every value read is
+ *     written earlier in the same call). Calls that overlap on the GPU (on
+ *     different streams, or from several threads) race on it: serialise them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int klein_block_forward_static(const klein_block_weights* w, void* x, int batch, int n_total, int row0, int rows,
+                               int n_txt, int n_img, const float* pos, const float* mod, void* stream);
+
 /* ------------------------------------------------------------------ model */
 
 /* All weights of a stack (device, borrowed; bf16 [out][in] unless noted).

@@ -74,6 +74,8 @@ _SIGS = {
     "klein_block_workspace_size": (c_size_t, [c_int, c_int]),
     "klein_block_forward": (c_int, [POINTER(KleinBlockWeights), c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                     c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "klein_block_forward_static": (c_int, [POINTER(KleinBlockWeights), c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                           c_int, c_void_p, c_void_p, c_void_p]),
     "klein_model_create": (c_int, [POINTER(c_void_p), POINTER(KleinModelDesc)]),
     "klein_model_destroy": (None, [c_void_p]),
     "klein_stack_workspace_size": (c_size_t, [POINTER(KleinSeq)]),
@@ -209,6 +211,17 @@ def klein_block_forward(w: dict, x, n_txt: int, n_img: int, pos, mod, ws, row0: 
     bw = block_weights(w)
     _check(lib.klein_block_forward(ctypes.byref(bw), _ptr(x), batch, n_total, row0, rows, n_txt, n_img, _ptr(pos),
                                    _ptr(mod), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def klein_block_forward_static(w: dict, x, n_txt: int, n_img: int, pos, mod, row0: int = 0,
+                               rows: int | None = None, stream=None):
+    """klein_block_forward with the library's fixed scratch instead of a
+    workspace (for callers that cannot allocate); batch * rows <= 256."""
+    batch, n_total = x.shape[0], x.shape[1]
+    rows = n_total - row0 if rows is None else rows
+    bw = block_weights(w)
+    _check(lib.klein_block_forward_static(ctypes.byref(bw), _ptr(x), batch, n_total, row0, rows, n_txt, n_img,
+                                          _ptr(pos), _ptr(mod), _stream(stream)))
 
 
 class KleinModel:

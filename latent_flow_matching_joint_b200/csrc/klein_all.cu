@@ -5,3 +5,4 @@
 #include "gemm.cu"
 #include "attention.cu"
 #include "klein_capi.cu"
+#include "static_ws.cu"

@@ -1,0 +1,75 @@
+"""The workspace-free block entry point, klein_block_forward_static.
+
+It serves callers that cannot allocate device memory (for example work
+recorded into a CUDA graph under global stream capture, where cudaMalloc is
+an error, or a plug-in that must not go around its host framework's memory
+pool): its scratch is a fixed array inside the library. Its results must
+match klein_block_forward with a caller workspace, call after call, since
+consecutive calls reuse (and inherit the contents of) the same array.
+
+Named so that pytest collects it last."""
+import ctypes
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import klein_inputs as ki  # noqa: E402
+from gpu_util import host, max_err_ratio, to_f32, upload_block, workspace  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from conftest import ensure_built
+    ensure_built()
+    import latent_flow_matching_joint_b200 as kb
+    return kb
+
+
+def test_static_scratch_block_matches_workspace_block(kb):
+    w = upload_block(ki.block_weights(0, "joint.0"))
+    n_txt, gh, gw = 80, 8, 8              # 80 text + 8x8 image tokens, batch 1
+    n = n_txt + gh * gw
+    x = ki.tokens(1, "no_alloc", 1, n)
+    mod = to_f32(ki.modulation_vectors(1, "no_alloc"))
+    pos = torch.empty((n, 4), dtype=torch.float32, device="cuda")
+    kb.klein_positions(kb.make_seq(1, n_txt, gh, gw), pos)
+
+    ref = to_f32(x)
+    ws = workspace(kb.klein_block_workspace_size(1, n))
+    kb.klein_block_forward(w, ref, n_txt, gh * gw, pos, mod, ws)
+    torch.cuda.synchronize()
+    expect = host(ref)
+
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    bw = kb.block_weights(w)
+    for call in range(2):                 # the second call reuses the first call's scratch
+        got = to_f32(x)
+        rc = kb.lib.klein_block_forward_static(ctypes.byref(bw), ctypes.c_void_p(got.data_ptr()), 1, n, 0, n, n_txt,
+                                               gh * gw, ctypes.c_void_p(pos.data_ptr()),
+                                               ctypes.c_void_p(mod.data_ptr()), stream)
+        assert rc == 0, kb.lib.klein_last_error()
+        torch.cuda.synchronize()
+        g = host(got)
+        assert np.all(np.isfinite(g)), call
+        assert max_err_ratio(g, expect) <= 2e-2, (call, max_err_ratio(g, expect))
+    assert kb.klein_device_status()[0] == 0
+
+
+def test_static_scratch_rejects_oversized_calls(kb):
+    w = upload_block(ki.block_weights(0, "joint.0"))
+    n = 300                               # 300 rows round up to 384 > 256
+    x = torch.zeros((1, n, ki.DIM), dtype=torch.float32, device="cuda")
+    pos = torch.zeros((n, 4), dtype=torch.float32, device="cuda")
+    mod = torch.zeros((3, 3, ki.DIM), dtype=torch.float32, device="cuda")
+    with pytest.raises(kb.KleinError) as e:
+        kb.klein_block_forward_static(w, x, 100, 200, pos, mod)
+    assert e.value.name == "KLEIN_ERR_WORKSPACE"
+    with pytest.raises(kb.KleinError) as e:   # batch 2 x 200 rows also exceeds it
+        kb.klein_block_forward_static(w, torch.zeros((2, 200, ki.DIM), device="cuda"), 100, 100, pos, mod)
+    assert e.value.name == "KLEIN_ERR_WORKSPACE"
