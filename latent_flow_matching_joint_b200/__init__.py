@@ -15,7 +15,7 @@ import os
 from ctypes import POINTER, Structure, c_float, c_int, c_longlong, c_size_t, c_uint, c_ulonglong, c_void_p
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "lib", "libklein.so")
+LIB_PATH = os.environ.get("KLEIN_LIB") or os.path.join(HERE, "lib", "libklein.so")
 
 DIM = 3072
 HEADS = 24
