@@ -326,6 +326,203 @@ static int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmAr
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
+// ---- CTA-pair variant: 256 x 256 output tiles per cluster of 2 CTAs.
+// Each CTA loads its 128 rows of A and its 128 rows of B (half the N tile) per
+// stage, so operand bytes per FLOP from L2 drop by a third against the
+// single-CTA 128 x 256 tile. The even CTA issues cta_group::2 MMAs
+// (M = 256, N = 256) that read both CTAs' shared memory and write each CTA's
+// 128 accumulator rows into its own tensor memory; its commits arrive on the
+// barriers of both CTAs. TMA completions of both CTAs are counted on the even
+// CTA's full barrier; both CTAs' epilogue threads release the accumulator on
+// the even CTA's empty barrier.
+
+struct PairCfg {
+  static constexpr int kStageA = 128 * 64 * 2;
+  static constexpr int kStageB = 128 * 64 * 2;
+  static constexpr int kStage = kStageA + kStageB;
+  static constexpr int kStages = 6;
+  static constexpr int kTileBytes = kStages * kStage;
+  static constexpr int kSmem = kTileBytes + 1024 + 256;
+  static constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
+  static constexpr int kThreads = 192;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                     const GemmArgs g) {
+  using Cfg = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kTileBytes);
+  uint64_t* empty = full + Cfg::kStages;
+  uint64_t* acc_full = empty + Cfg::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 256);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barrier initialisation and the TMEM allocation are visible pair-wide
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = g.batch * g.m_tiles_per_b;
+  const int total = m_tiles * g.n_tiles;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  constexpr uint32_t idesc = idesc_bf16_f32(256, 256);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < total; tile += npairs) {
+        const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
+        const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
+        const int b = m_idx / g.m_tiles_per_b;
+        const int row0 = (m_idx % g.m_tiles_per_b) * 256 + 128 * static_cast<int>(rank);
+        int brow;
+        if (EPI == kEpiQKV && n_idx >= g.b_split) {
+          const int chunk = n_idx - g.b_split;
+          brow = (leader ? 3 * kDim : 3 * kDim + kMlp) + chunk * 128;
+        } else {
+          brow = n_idx * 256 + 128 * static_cast<int>(rank);
+        }
+        bool ok = true;
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, 0x111)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStage);
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          uint8_t* sa = smem + stage * Cfg::kStage;
+          tma_load_3d_pair(sa, &map_a, bar, kb * 64, row0, b);
+          tma_load_2d_pair(sa + Cfg::kStageA, &map_b, bar, kb * 64, brow);
+          if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int tile = pair; tile < total; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, 0x112)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * 256;
+        bool ok = true;
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, 0x113)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * Cfg::kStage);
+          const uint32_t b0 = a0 + Cfg::kStageA;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, (kb | k) != 0);
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&acc_full[acc], 0x3);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int rloc = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++it) {
+      const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
+      const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
+      const int b = m_idx / g.m_tiles_per_b;
+      const int r = (m_idx % g.m_tiles_per_b) * 256 + 128 * static_cast<int>(rank) + rloc;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&acc_full[acc], acc_phase, 0x114)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + acc * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (EPI == kEpiF32) epi_store<256>(taddr, g, b, r, n_idx, true);
+      else if (EPI == kEpiQKV) epi_qkv(taddr, g, b, r, n_idx);
+      else epi_resid<256>(taddr, g, b, r, n_idx);
+      tc_fence_before();
+      mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // every pair MMA and every epilogue of both CTAs is done
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int EPI>
+static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
+  using Cfg = PairCfg;
+  static int max_pairs = 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs == 0) {
+    if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+        cudaSuccess)
+      return -1;
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<EPI>, &cfg) != cudaSuccess || n < 1) return -1;
+    max_pairs = n;
+  }
+  const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
+  if (total <= 0) return 0;
+  const int pairs = total < max_pairs ? total : max_pairs;
+  cfg.gridDim = dim3(2 * pairs);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, ma, mb, g);
+  note_launch();
+  return e == cudaSuccess ? 0 : -1;
+}
+
+int launch_gemm_pair(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
+  switch (epi) {
+    case kEpiF32: return launch_pair_one<kEpiF32>(ma, mb, g, s);
+    case kEpiQKV: return launch_pair_one<kEpiQKV>(ma, mb, g, s);
+    case kEpiResid: return launch_pair_one<kEpiResid>(ma, mb, g, s);
+  }
+  return -2;
+}
+
 int launch_gemm(int bn, int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
                 cudaStream_t s) {
   if (bn == 256) {

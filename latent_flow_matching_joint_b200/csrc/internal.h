@@ -60,6 +60,10 @@ struct GemmArgs {
 };
 
 // C[M,N] = A[M,K] * B[N,K]^T with epilogue `epi`; bn = 128 or 256.
+// Same product on CTA pairs (clusters of 2) with 256 x 256 tiles: args.m_tiles_per_b
+// counts 256-row tiles, args.n_tiles 256-column tiles; epi is kEpiF32, kEpiQKV or kEpiResid.
+int launch_gemm_pair(int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
+                     cudaStream_t stream);
 int launch_gemm(int bn, int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
                 cudaStream_t stream);
 

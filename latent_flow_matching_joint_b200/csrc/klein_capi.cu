@@ -153,6 +153,18 @@ static BlockWs carve_block(void* base, int batch, int rows) {
 
 // ------------------------------------------------------------------ block
 
+// The block's two big GEMMs run on CTA pairs (256 x 256 tiles) unless the
+// library is built with KLEIN_GEMM_PAIR=0 (single CTAs, 128 x 256 tiles).
+#ifndef KLEIN_GEMM_PAIR
+#define KLEIN_GEMM_PAIR 1
+#endif
+constexpr int kGemmRowsPerTile = KLEIN_GEMM_PAIR ? 256 : 128;
+
+static int launch_block_gemm(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                             cudaStream_t s) {
+  return KLEIN_GEMM_PAIR ? launch_gemm_pair(epi, ma, mb, g, s) : launch_gemm(256, epi, ma, mb, g, s);
+}
+
 // One block over rows [row0, row0+rows) of x. `rope` holds the view's table
 // (row 0 = global row row0). Workspace `w` is carved for (batch, >= rows).
 static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_total, int row0, int rows,
@@ -180,7 +192,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   GemmArgs g{};
   g.batch = batch;
   g.rows = rows;
-  g.m_tiles_per_b = (rows + 127) / 128;
+  g.m_tiles_per_b = (rows + kGemmRowsPerTile - 1) / kGemmRowsPerTile;
   g.n_tiles = 36 + kMlp / 128;
   g.k_blocks = kDim / 64;
   g.b_split = 36;
@@ -193,7 +205,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   g.rope = rope;
   g.rows_pad = rp;
   pi = prof_begin(kProfGemmIn, s);
-  if (launch_gemm(256, kEpiQKV, m_h, m_win, g, s)) return cuda_fail("in-projection GEMM launch");
+  if (launch_block_gemm(kEpiQKV, m_h, m_win, g, s)) return cuda_fail("in-projection GEMM launch");
   prof_end(pi, s);
   // a6: attention
   AttnArgs at{};
@@ -211,7 +223,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   GemmArgs o{};
   o.batch = batch;
   o.rows = rows;
-  o.m_tiles_per_b = (rows + 127) / 128;
+  o.m_tiles_per_b = (rows + kGemmRowsPerTile - 1) / kGemmRowsPerTile;
   o.n_tiles = kDim / 256;
   o.k_blocks = kOutK / 64;
   o.n_fastest = 1;
@@ -222,7 +234,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   o.n_txt = n_txt;
   o.n_img = n_img;
   pi = prof_begin(kProfGemmOut, s);
-  if (launch_gemm(256, kEpiResid, m_aout, m_wout, o, s)) return cuda_fail("out-projection GEMM launch");
+  if (launch_block_gemm(kEpiResid, m_aout, m_wout, o, s)) return cuda_fail("out-projection GEMM launch");
   prof_end(pi, s);
   return KLEIN_OK;
 }
@@ -719,17 +731,22 @@ int klein_op_gemm(const void* a, const void* b, float* c, int m, int n, int k, v
   if (make_map_3d(&ma, a, k, m, 1, (uint64_t)k * 2, (uint64_t)m * k * 2, 64, 128) ||
       make_map_2d(&mb, b, k, n, (uint64_t)k * 2, 64, 128))
     return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-  const int bn = (n % 256 == 0) ? 256 : 128;
+  // N a multiple of 256: the block GEMM configuration (CTA pairs unless
+  // built without them); otherwise single CTAs with 128-column tiles.
+  const bool wide = (n % 256) == 0;
+  const int rows_per_tile = wide ? kGemmRowsPerTile : 128;
   GemmArgs g{};
   g.batch = 1;
   g.rows = m;
-  g.m_tiles_per_b = (m + 127) / 128;
-  g.n_tiles = n / bn;
+  g.m_tiles_per_b = (m + rows_per_tile - 1) / rows_per_tile;
+  g.n_tiles = n / (wide ? 256 : 128);
   g.k_blocks = k / 64;
   g.out = c;
   g.out_ld = n;
   g.out_bstride = m;
-  if (launch_gemm(bn, kEpiF32, ma, mb, g, static_cast<cudaStream_t>(stream))) return cuda_fail("gemm launch");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rc = wide ? launch_block_gemm(kEpiF32, ma, mb, g, s) : launch_gemm(128, kEpiF32, ma, mb, g, s);
+  if (rc) return cuda_fail("gemm launch");
   return KLEIN_OK;
 }
 
