@@ -28,12 +28,6 @@
 #include "common.cuh"
 #include "internal.h"
 
-// One probability pair in KLEIN_ATTN_POLY_EVERY is exponentiated on the FMA
-// pipe (0 = all on MUFU).
-#ifndef KLEIN_ATTN_POLY_EVERY
-#define KLEIN_ATTN_POLY_EVERY 0
-#endif
-
 namespace klein {
 
 namespace {
@@ -46,25 +40,6 @@ constexpr int kSmem = kOffBar + 256 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only when the max grows by > 2^8
-
-// 2^x on the FMA pipe, for x in [-125, 9]: n = round(x) by the 1.5 * 2^23
-// addition trick, f = x - n in [-1/2, 1/2], 2^f by a cubic fitted for minimum
-// maximum relative error (csrc/fit_exp2_poly.py: 7.5e-5 in float32 Horner
-// form, far below the bf16 rounding of P), and 2^n added to the exponent
-// bits. Off by default: measured on B200 at 4608 and 2 x 16944 rows, moving
-// a quarter or an eighth of the exponentials here was 4-6 % slower than
-// MUFU alone (the softmax is latency-bound, not MUFU-bound).
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -125.0f);
-  const float kShifter = 12582912.0f;  // 1.5 * 2^23
-  const float t = x + kShifter;
-  const float f = x - (t - kShifter);
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  // the low bits of t hold n (two's complement); shifted into the exponent field
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -200,20 +175,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : -INFINITY;
       }
-      // row max as a tree of independent partial maxima
-      float m4[8];
+      // row max: 8 independent chains of three-input maxima
+      float m8[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) m4[q] = s[q];
+      for (int q = 0; q < 8; ++q) m8[q] = fmax3(s[q], s[q + 8], s[q + 16]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) m4[i & 7] = fmaxf(m4[i & 7], s[i]);
+      for (int i = 24; i < 120; i += 16) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], m4[q + 4]);
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        for (int q = 0; q < 8; ++q) m8[q] = fmax3(m8[q], s[i + q], s[i + 8 + q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], s[120 + q]);
+      const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
       const float m_cand = mx * sl2;
       // move the running max only if it grows past the threshold
       const bool grow = m_cand > m_run + kRescaleThreshold;
       const float m_new = grow ? m_cand : m_run;
       const float alpha = fast_exp2(m_run - m_new);
+      // p = exp2(s * scale - m): the affine step two lanes per instruction,
+      // exp2 on MUFU, sums two-wide in four independent accumulators
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {  // masked keys: exp2(-inf) = 0 exactly
+        float x0, x1;
+        ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -m_new, -m_new);
+        const float p0 = fast_exp2(x0);
+        const float p1 = fast_exp2(x1);
+        fadd2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
+        pk[i >> 1] = pack_bf16(p0, p1);
+      }
+      float sum4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sum4[q] = sa[q] + sb[q];
+      // rescale the output row after the scores are consumed, so that the
+      // scores and an output chunk are never live together
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         float o[32];
 #pragma unroll 1
@@ -222,29 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
           tmem_st32(o_col + 32 * c, o);
-        }
-      }
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
-      if (!tail) {
-#pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          const float x0 = fmaf(s[i], sl2, -m_new);
-          const float x1 = fmaf(s[i + 1], sl2, -m_new);
-          // one pair in KLEIN_ATTN_POLY_EVERY on the FMA pipe, the rest on MUFU
-          const bool on_fma = KLEIN_ATTN_POLY_EVERY > 0 && ((i >> 1) % (KLEIN_ATTN_POLY_EVERY > 0 ? KLEIN_ATTN_POLY_EVERY : 1)) == KLEIN_ATTN_POLY_EVERY - 1;
-          const float p0 = on_fma ? poly_exp2(x0) : fast_exp2(x0);
-          const float p1 = on_fma ? poly_exp2(x1) : fast_exp2(x1);
-          sum4[(i >> 1) & 3] += p0 + p1;
-          pk[i >> 1] = pack_bf16(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; i += 2) {  // masked keys: exp2(-inf) = 0 exactly on MUFU
-          const float p0 = fast_exp2(fmaf(s[i], sl2, -m_new));
-          const float p1 = fast_exp2(fmaf(s[i + 1], sl2, -m_new));
-          sum4[(i >> 1) & 3] += p0 + p1;
-          pk[i >> 1] = pack_bf16(p0, p1);
         }
       }
       l_run = l_run * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
@@ -294,7 +267,7 @@ int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   dim3 grid((a.rows + 255) / 256, a.heads, a.batch);
   attn_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mvt, a);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 }  // namespace klein

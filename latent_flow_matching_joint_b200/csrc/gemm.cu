@@ -323,7 +323,7 @@ static int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmAr
   const int grid = total < num_sms() ? total : num_sms();
   gemm_kernel<BN, EPI><<<grid, Cfg::kThreads, Cfg::kSmem, s>>>(ma, mb, g);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ---- CTA-pair variant: 256 x 256 output tiles per cluster of 2 CTAs.
@@ -511,7 +511,7 @@ static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const G
   cfg.gridDim = dim3(2 * pairs);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, ma, mb, g);
   note_launch();
-  return e == cudaSuccess ? 0 : -1;
+  return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 int launch_gemm_pair(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {

@@ -71,7 +71,7 @@ int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16*
   modln_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, h, batch, rows, n_txt, n_img, mod, mod_stride,
                                       single_mode);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // bf16 rows -> fp32 rows of the residual stream: src [batch][rows][3072]
@@ -101,7 +101,7 @@ int launch_rows_to_f32(const __nv_bfloat16* src, long long src_bstride, float* d
                                                                   reinterpret_cast<float4*>(dst), dst_bstride,
                                                                   dst_row0, rows, total);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ RoPE
@@ -129,7 +129,7 @@ int launch_rope_table(const float* pos, float2* table, int rows, float theta, cu
   if (n <= 0) return 0;
   rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(pos, table, rows, static_cast<double>(theta));
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // Standalone rotation of [rows][heads][128] bf16 (the same arithmetic as the
@@ -162,7 +162,7 @@ int launch_rope_apply(const __nv_bfloat16* in, __nv_bfloat16* out, const float2*
   rope_apply_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out),
                                            table, rows, heads);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ positions
@@ -217,7 +217,7 @@ int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, co
   if (total <= 0) return 0;
   positions_kernel<<<(total + 255) / 256, 256, 0, s>>>(pos, n_txt, img_h, img_w, rd, total);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ Euler + CFG
@@ -253,7 +253,7 @@ int launch_euler(float* x, const float* vc, const float* vu, long long n, float 
                                       reinterpret_cast<const float4*>(vu), n4, dsigma, g,
                                       reinterpret_cast<float4*>(x0), sigma);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 __global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, long long n4) {
@@ -269,7 +269,7 @@ int launch_to_bf16(const float* in, __nv_bfloat16* out, long long n, cudaStream_
   to_bf16_kernel<<<(int)((n4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(in),
                                                          reinterpret_cast<uint2*>(out), n4);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ GEMV
@@ -331,7 +331,7 @@ int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_
   }
   gemv_kernel<<<(n_out + 7) / 8, 256, smem, s>>>(w, n_out, k, x, n_vec, x_stride, y, y_stride, act_silu, add);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ time embedding + modulation
@@ -411,7 +411,7 @@ __global__ void wait_probe_kernel(unsigned long long limit_ns) {
 int launch_wait_probe(unsigned long long limit_ns, cudaStream_t s) {
   wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 }  // namespace klein
