@@ -41,6 +41,14 @@ WORKLOADS = {
 }
 
 
+# dram__bytes_read.sum + dram__bytes_write.sum of the in-projection GEMM
+# (gemm_pair_kernel<2>), mean over the first 42 launches of a t2i denoise, from
+# one ncu capture of the current kernel (its summary is kept with the other
+# kernel profiles). Must be re-captured (or set to None) whenever that kernel
+# changes.
+GEMM_IN_TRAFFIC_BYTES = 314.35e6
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -360,7 +368,9 @@ def run_ours(args):
     achieved = gi_flops / (gi_ms / 1e3) / 1e12 if gi_ms > 0 else 0.0
     roofline = {"kernel": "gemm_in (fused QKV + MLP-in, tcgen05)", "bound": "tensor", "achieved": achieved,
                 "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
-                "traffic": None, "avg_launch_ms": gi_avg_ms, "launches": gi_n,
+                "traffic": GEMM_IN_TRAFFIC_BYTES if args.workload == "t2i" else None,
+                "traffic_unit": "bytes per launch (ncu dram read + write)",
+                "avg_launch_ms": gi_avg_ms, "launches": gi_n,
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
 
     # ---- end to end through the public API with host buffers
