@@ -86,6 +86,24 @@ def gemm_in_rows_per_step(n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
     return n_stage1 * (n_txt + n_img + n_ref) + n_joint * (n_txt + n_img + n_ref)
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's duration; every rank must call this (a collective)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank processed units_per_rank within ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -346,16 +364,12 @@ def run_ours(args):
     barrier()
     prof = kb.klein_profile_end()
     gpu_launches = kb.klein_launch_count() - launches0
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     rc, site, msg = kb.klein_device_status()
     if rc != 0:
         raise RuntimeError(f"device error in the timed region: {msg}")
     ms_per_image = ms / args.steps
-    value = world * steps * args.steps / (ms / 1e3)
+    value = job_rate(world, steps * args.steps, ms)
     f_step = step_flops(batch, n_txt, n_img, n_ref)
     peaks = load_peaks()
 
@@ -397,14 +411,10 @@ def run_ours(args):
         e2e_image()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = noise_h.numel() * 4 + text_h.numel() * 2 + (ref_h.numel() * 4 if n_ref else 0)
     d2h = out_h.numel() * 4
-    e2e = {"value": world * steps * args.steps / (ms_e2e / 1e3), "unit": "denoise steps/s",
+    e2e = {"value": job_rate(world, steps * args.steps, ms_e2e), "unit": "denoise steps/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "note": "per bench step (one image): pinned host noise + text (+ reference) -> device, klein_denoise, "
                    "final latents -> host"}
