@@ -85,6 +85,31 @@ def test_block_matches_oracle(kb, weights, name):
     assert max_err_ratio(d_got, d_ref) <= 0.1
 
 
+@pytest.mark.parametrize("batch,n_txt,grid,refs", [
+    (1, 512, (64, 64), ((64, 64),)),     # 1024x1024 edit: 512 + 4096 + 4096 = 8704 tokens
+    (2, 560, (128, 128), ()),            # 2048x2048 base with guidance: 2 x (560 + 16384) = 2 x 16944
+])
+def test_block_large_sampled_rows(kb, weights, batch, n_txt, grid, refs):
+    # full-size joint blocks of the edit and 2048x2048 workloads; the oracle
+    # evaluates a sample of output rows (every row supplies keys and values)
+    w, wd = weights
+    n_img = grid[0] * grid[1]
+    n_ref = sum(h * ww for h, ww in refs)
+    n_total = n_txt + n_img + n_ref
+    seq = kb.make_seq(batch, n_txt, grid[0], grid[1], refs)
+    x = ki.tokens(1, f"block.large.{n_total}", batch, n_total)
+    mod = ki.modulation_vectors(1, f"block.large.{n_total}")
+    got = run_block(kb, wd, x, seq, mod, 0, n_total, n_txt, n_img)
+    rows = np.unique(np.concatenate([np.arange(0, n_total, 997), [0, n_txt - 1, n_txt, n_txt + n_img,
+                                                                 n_total - 1]]))
+    ref = o.block(x, o.positions(n_txt, grid, refs), o.mode_of_rows(n_txt, n_img, n_ref),
+                  mod.astype(np.float64), w, rows=rows)
+    g = got[:, rows]
+    assert np.all(np.isfinite(g))
+    assert max_err_ratio(g, ref) <= 2e-2, max_err_ratio(g, ref)
+    assert cosine(g - x[:, rows], ref - x[:, rows]) >= 0.999
+
+
 def test_block_config2_sampled_rows(kb, weights):
     # 1024x1024 text-to-image joint block: 512 text + 64x64 image, batch 1;
     # the oracle computes a sample of output rows (all rows give keys/values).

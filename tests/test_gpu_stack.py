@@ -140,3 +140,30 @@ def test_denoise_argument_errors(kb, base):
         kb.klein_stack_forward(model, x, to_bf16(text), x, 0.5, 0.0, seq_r,
                                torch.empty((1, 4, 128), device="cuda"), workspace(kb.klein_stack_workspace_size(seq_r)))
     assert e.value.name == "KLEIN_ERR_INVALID_ARG"
+
+
+def test_full_depth_denoise_matches_stored_oracle(kb):
+    """The full 5 + 28 block distilled stack, 16 Euler steps, 80 text + 8x8
+    image tokens: final latents against the oracle's, stored by
+    tests/golden/make_denoise_golden.py (cosine >= 0.999)."""
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    path = os.path.join(here, "denoise_full_depth_80_8x8_16.npy")
+    meta = json.load(open(path.replace(".npy", ".json")))
+    m = ki.ModelWeights(seed=meta["weight_seed"], distilled=True)
+    t = upload_model(m, with_ref=False)
+    m._blocks.clear()
+    model = kb.KleinModel(t)
+    n_txt, (gh, gw) = meta["n_txt"], meta["grid"]
+    seq = kb.make_seq(1, n_txt, gh, gw)
+    x = to_f32(ki.noise_latents(meta["noise_seed"], gh * gw))
+    text = to_bf16(ki.text_embeddings(meta["text_seed"], 1, n_txt))
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, text, None, meta["steps"], 1.0, seq, ws)
+    torch.cuda.synchronize()
+    ref = np.load(path)
+    got = host(x)
+    assert np.all(np.isfinite(got))
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)
