@@ -102,6 +102,7 @@ def test_block_large_sampled_rows(kb, weights, batch, n_txt, grid, refs):
     got = run_block(kb, wd, x, seq, mod, 0, n_total, n_txt, n_img)
     rows = np.unique(np.concatenate([np.arange(0, n_total, 997), [0, n_txt - 1, n_txt, n_txt + n_img,
                                                                  n_total - 1]]))
+    rows = rows[rows < n_total]
     ref = o.block(x, o.positions(n_txt, grid, refs), o.mode_of_rows(n_txt, n_img, n_ref),
                   mod.astype(np.float64), w, rows=rows)
     g = got[:, rows]
