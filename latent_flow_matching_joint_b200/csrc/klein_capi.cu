@@ -570,15 +570,27 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
   };
   if ((rc = project(latents, n_img, d.img_in, n_txt))) return rc;
   if (n_ref && (rc = project(refs, n_ref, d.ref_in, n_txt + n_img))) return rc;
-  // a8 stage 1: each stream through its own blocks, attending to itself
+  // a8 stage 1: each stream through its own blocks, attending to itself.
+  // The image and reference streams start from the same latents in every
+  // batch item (the batch only varies the text, e.g. guidance's cond and
+  // uncond prompts) and stage 1 never mixes streams, so they are computed
+  // for batch item 0 and copied to the others.
   const int lo[3] = {0, n_txt, n_txt + n_img};
   const int cnt[3] = {n_txt, n_img, n_ref};
   for (int md = 0; md < 3; ++md) {
     if (cnt[md] == 0) continue;
+    const int nb = md == 0 ? B : 1;
     for (int i = 0; i < d.n_stage1; ++i) {
-      rc = block_impl(&d.stage1[md][i], w.x, B, n_total, lo[md], cnt[md], n_txt, n_img,
+      rc = block_impl(&d.stage1[md][i], w.x, nb, n_total, lo[md], cnt[md], n_txt, n_img,
                       w.rope + (size_t)lo[md] * kPairs, w.mod, w.blk, s);
       if (rc) return rc;
+    }
+  }
+  if (d.n_stage1 > 0) {
+    for (int b = 1; b < B; ++b) {
+      if (cudaMemcpyAsync(w.x + ((size_t)b * n_total + n_txt) * kDim, w.x + (size_t)n_txt * kDim,
+                          (size_t)(n_img + n_ref) * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return cuda_fail("stage-1 stream copy");
     }
   }
   // a8 stage 2: joint blocks over everything

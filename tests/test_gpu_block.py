@@ -88,6 +88,8 @@ def test_block_matches_oracle(kb, weights, name):
 @pytest.mark.parametrize("batch,n_txt,grid,refs", [
     (1, 512, (64, 64), ((64, 64),)),     # 1024x1024 edit: 512 + 4096 + 4096 = 8704 tokens
     (2, 560, (128, 128), ()),            # 2048x2048 base with guidance: 2 x (560 + 16384) = 2 x 16944
+    (1, 512, (256, 256), ()),            # the largest output, 4096x4096: 512 + 65536 tokens
+    (3, 160, (16, 16), ((8, 8), (4, 6))),  # batch 3, two references
 ])
 def test_block_large_sampled_rows(kb, weights, batch, n_txt, grid, refs):
     # full-size joint blocks of the edit and 2048x2048 workloads; the oracle
