@@ -53,8 +53,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* kv_empty = bars + 5;  // [2]
   uint64_t* s_full = bars + 7;    // [2 tiles]: scores ready (phase j), final output ready (phase nkv)
-  uint64_t* p_full = bars + 9;    // [2 tiles]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* p_full = bars + 9;    // [2 tiles][2 halves of the keys]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[2 * s], 128);
+      mbar_init(&p_full[2 * s + 1], 128);
     }
     fence_barrier_init();
     tma_prefetch_desc(&map_q);
@@ -129,16 +130,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nkv; ++j) {
         const int st = j & 1;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait(&p_full[t], j & 1, 0x204)) { ok = false; break; }
           if (t == 0 && !mbar_wait(&v_full[st], (j >> 1) & 1, 0x205)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t v0 = smem_u32(smem + kOffV + st * kTileBytes);
+          for (int half = 0; half < 2; ++half) {
+            if (!mbar_wait(&p_full[2 * t + half], j & 1, 0x204)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-            umma_bf16_tmem_a(tmem_base + t * 256 + 128, tmem_base + t * 256 + kk * 8, sw128_desc(v0 + off), idesc,
-                             (j | kk) != 0);
+            for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
+              const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+              umma_bf16_tmem_a(tmem_base + t * 256 + 128, tmem_base + t * 256 + kk * 8, sw128_desc(v0 + off),
+                               idesc, (j | kk) != 0);
+            }
           }
+          if (!ok) break;
           if (t == 1) umma_commit(&kv_empty[st]);
           if (j + 1 < nkv) {
             if (t == 0) {
@@ -193,38 +197,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = grow ? m_cand : m_run;
       const float alpha = fast_exp2(m_run - m_new);
       // p = exp2(s * scale - m): the affine step two lanes per instruction,
-      // exp2 on MUFU, sums two-wide in four independent accumulators
+      // exp2 on MUFU, sums two-wide in four independent accumulators. P goes
+      // back to TMEM in two halves of 64 keys, each released to the MMA warp
+      // on its own barrier, so O += P V over the first half runs while the
+      // second half is being exponentiated.
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {  // masked keys: exp2(-inf) = 0 exactly
-        float x0, x1;
-        ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -m_new, -m_new);
-        const float p0 = fast_exp2(x0);
-        const float p1 = fast_exp2(x1);
-        fadd2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
-        pk[i >> 1] = pack_bf16(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int i = 64 * half; i < 64 * half + 64; i += 2) {  // masked keys: exp2(-inf) = 0 exactly
+          float x0, x1;
+          ffma2(x0, x1, s[i], s[i + 1], sl2, sl2, -m_new, -m_new);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          fadd2(sa[(i >> 1) & 3], sb[(i >> 1) & 3], p0, p1);
+          pk[(i >> 1) & 31] = pack_bf16(p0, p1);
+        }
+        // the output row is rescaled (rarely) before any P V of this key
+        // tile is released, and after half the scores are consumed
+        if (half == 0 && j > 0 && __any_sync(0xffffffffu, grow)) {
+          float o[32];
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(o_col + 32 * c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(o_col + 32 * c, o);
+          }
+        }
+        tmem_st32(s_col + 32 * half, reinterpret_cast<const float*>(pk));
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * t + half]);
       }
       float sum4[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) sum4[q] = sa[q] + sb[q];
-      // rescale the output row after the scores are consumed, so that the
-      // scores and an output chunk are never live together
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        float o[32];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(o_col + 32 * c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(o_col + 32 * c, o);
-        }
-      }
       l_run = l_run * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m_run = m_new;
-      tmem_st64(s_col, pk);
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
     }
     if (ok && mbar_wait(&s_full[t], nkv & 1, 0x208)) {
       tc_fence_after();
