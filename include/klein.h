@@ -213,6 +213,10 @@ typedef struct {
   const void* mod[2][3];   /* [9216][3072] per stage (1, 2) and stream: (shift, scale, gate) */
   const void* final_mod;   /* [6144][3072] final (shift, scale) */
   const void* final_out;   /* [128][3072] output projection to latent channels */
+  const void* txt_in;      /* [3072][20480] text input projection, or NULL. The text encoder's
+                              hidden states from eight of its layers, 2560 wide each, stacked to
+                              20480 per token ([blog]; [guide] "The text encoder"), are projected to
+                              the model width. NULL: text is given already at 3072. */
 } klein_model_desc;
 
 typedef struct klein_model klein_model;
@@ -233,7 +237,10 @@ size_t klein_stack_workspace_size(const klein_seq* seq);
  * [text | image | reference]; the image rows then pass the final modulated
  * LayerNorm and projection to 128 channels.
  *   latents  device float [n_img][128], shared by the batch
- *   text     device bf16 [batch][n_txt][3072]
+ *   text     device bf16 [batch][n_txt][3072], or [batch][n_txt][20480] (the
+ *            stacked encoder layers) when the model has txt_in; the
+ *            projection runs once per klein_denoise call (text does not
+ *            change across steps)
  *   refs     device float [n_ref][128] or NULL when seq->n_refs == 0
  *   v_out    device float [batch][n_img][128]
  *   ws       device workspace >= klein_stack_workspace_size(seq) */

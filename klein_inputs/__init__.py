@@ -96,8 +96,12 @@ def block_name(stage: int, mode: str | None, index: int) -> str:
     return f"joint.{index}"
 
 
-def misc_weights(seed: int, distilled: bool) -> dict:
-    """Everything that is not a block: embedders, modulation, in/out layers."""
+TEXT_STACK = 8 * 2560  # eight encoder layers of width 2560, stacked per text token
+
+
+def misc_weights(seed: int, distilled: bool, txt_in: bool = False) -> dict:
+    """Everything that is not a block: embedders, modulation, in/out layers
+    (txt_in: also the 20480 -> 3072 text input projection)."""
     w = {
         "img_in": linear(seed, "img_in", DIM, LATENT_CH),
         "ref_in": linear(seed, "ref_in", DIM, LATENT_CH),
@@ -112,6 +116,8 @@ def misc_weights(seed: int, distilled: bool) -> dict:
     if distilled:
         w["tt_mlp1"] = linear(seed, "tt_mlp1", DIM, TIME_FREQ_DIM)
         w["tt_mlp2"] = linear(seed, "tt_mlp2", DIM, DIM)
+    if txt_in:
+        w["txt_in"] = linear(seed, "txt_in", DIM, TEXT_STACK)
     return w
 
 
@@ -123,18 +129,19 @@ class ModelWeights:
     """
 
     def __init__(self, seed: int = WEIGHT_SEED, distilled: bool = True,
-                 n_stage1: int = N_STAGE1, n_joint: int = N_JOINT):
+                 n_stage1: int = N_STAGE1, n_joint: int = N_JOINT, txt_in: bool = False):
         self.seed = seed
         self.distilled = distilled
         self.n_stage1 = n_stage1
         self.n_joint = n_joint
+        self.txt_in = txt_in
         self._blocks: dict = {}
         self._misc = None
 
     @property
     def misc(self) -> dict:
         if self._misc is None:
-            self._misc = misc_weights(self.seed, self.distilled)
+            self._misc = misc_weights(self.seed, self.distilled, self.txt_in)
         return self._misc
 
     def block(self, stage: int, mode: str | None, index: int) -> dict:
@@ -162,6 +169,11 @@ def tokens(seed: int, tag: str, batch: int, rows: int) -> np.ndarray:
 def text_embeddings(seed: int, batch: int, n_txt: int) -> np.ndarray:
     """Text-encoder output stand-in [batch, n_txt, DIM]; batch 2 = cond, uncond."""
     return normal(seed, "text_emb", (batch, n_txt, DIM))
+
+
+def text_hidden_states(seed: int, batch: int, n_txt: int) -> np.ndarray:
+    """Stacked text-encoder hidden states stand-in [batch, n_txt, 20480], N(0,1)."""
+    return normal(seed, "text_hidden", (batch, n_txt, TEXT_STACK))
 
 
 def noise_latents(seed: int, n_img: int) -> np.ndarray:

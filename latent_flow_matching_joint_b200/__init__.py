@@ -55,7 +55,7 @@ class KleinModelDesc(Structure):
     _fields_ = [("n_stage1", c_int), ("n_joint", c_int), ("stage1", c_void_p * 3), ("joint", c_void_p),
                 ("img_in", c_void_p), ("ref_in", c_void_p), ("t_mlp1", c_void_p), ("t_mlp2", c_void_p),
                 ("tt_mlp1", c_void_p), ("tt_mlp2", c_void_p), ("mod", (c_void_p * 3) * 2),
-                ("final_mod", c_void_p), ("final_out", c_void_p)]
+                ("final_mod", c_void_p), ("final_out", c_void_p), ("txt_in", c_void_p)]
 
 
 _SIGS = {
@@ -250,7 +250,8 @@ class KleinModel:
         self._joint = (KleinBlockWeights * max(1, len(joint)))(*[block_weights(b) for b in joint])
         d.joint = ctypes.cast(self._joint, c_void_p) if joint else None
         g = tensors.get
-        for name in ("img_in", "ref_in", "t_mlp1", "t_mlp2", "tt_mlp1", "tt_mlp2", "final_mod", "final_out"):
+        for name in ("img_in", "ref_in", "t_mlp1", "t_mlp2", "tt_mlp1", "tt_mlp2", "final_mod", "final_out",
+                     "txt_in"):
             t = g(name)
             setattr(d, name, t.data_ptr() if t is not None else None)
         for s in (0, 1):

@@ -269,6 +269,7 @@ struct StackWs {
   float* tscratch;   // 8 * 3072 floats
   __nv_bfloat16* lat_bf;  // [max(n_img, n_ref)][128]
   float* v;          // [batch][n_img][128]
+  float* txt;        // [batch][n_txt][3072] projected text (models with txt_in)
   BlockWs blk;
   size_t bytes;
 };
@@ -289,6 +290,7 @@ static StackWs carve_stack(void* base, int batch, int n_total, int n_img, int n_
   w.tscratch = reinterpret_cast<float*>(take((size_t)8 * kDim * sizeof(float)));
   w.lat_bf = reinterpret_cast<__nv_bfloat16*>(take((size_t)(n_img > n_ref ? n_img : n_ref) * kLatent * 2));
   w.v = reinterpret_cast<float*>(take((size_t)batch * n_img * kLatent * sizeof(float)));
+  w.txt = reinterpret_cast<float*>(take((size_t)batch * (n_total - n_img - n_ref) * kDim * sizeof(float)));
   w.blk = carve_block(base ? static_cast<char*>(base) + off : nullptr, batch, n_total);
   off += w.blk.bytes;
   w.bytes = off;
@@ -307,7 +309,7 @@ extern "C" {
 
 const char* klein_last_error(void) { return g_msg; }
 
-int klein_version(void) { return 100; }
+int klein_version(void) { return 101; }
 
 long long klein_launch_count(void) { return g_launches; }
 
@@ -483,6 +485,7 @@ int klein_model_create(klein_model** out, const klein_model_desc* d) {
       if (!d->mod[st][m]) return fail(KLEIN_ERR_INVALID_ARG, "modulation weights incomplete");
   if ((d->tt_mlp1 == nullptr) != (d->tt_mlp2 == nullptr))
     return fail(KLEIN_ERR_INVALID_ARG, "target embedder needs both layers");
+  if (d->txt_in && !aligned16(d->txt_in)) return fail(KLEIN_ERR_ALIGN, "txt_in must be 16-byte aligned");
   klein_model* m = new (std::nothrow) klein_model;
   if (!m) return fail(KLEIN_ERR_INVALID_ARG, "out of host memory");
   m->d = *d;
@@ -522,27 +525,61 @@ int klein_op_time_mod(const klein_model* m, float sigma, float sigma_next, int w
   return KLEIN_OK;
 }
 
+constexpr int kTextStack = 8 * 2560;  // eight 2560-wide encoder layers per text token
+
+// Text input projection (models with txt_in): w.txt = text [B][n_txt][20480] x txt_in^T.
+static int project_text(const klein_model* m, const void* text, const klein_seq* seq, const StackWs& w,
+                        cudaStream_t s) {
+  const int B = seq->batch;
+  const int n_txt = seq->n_txt;
+  CUtensorMap ma, mb;
+  if (make_map_3d(&ma, text, kTextStack, n_txt, B, (uint64_t)kTextStack * 2, (uint64_t)n_txt * kTextStack * 2, 64,
+                  128) ||
+      make_map_2d(&mb, m->d.txt_in, kTextStack, kDim, (uint64_t)kTextStack * 2, 64, 128))
+    return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  GemmArgs g{};
+  g.batch = B;
+  g.rows = n_txt;
+  g.m_tiles_per_b = (n_txt + kGemmRowsPerTile - 1) / kGemmRowsPerTile;
+  g.n_tiles = kDim / 256;
+  g.k_blocks = kTextStack / 64;
+  g.out = w.txt;
+  g.out_ld = kDim;
+  g.out_bstride = n_txt;
+  const int pi = prof_begin(kProfProj, s);
+  if (launch_block_gemm(kEpiF32, ma, mb, g, s)) return cuda_fail("text projection launch");
+  prof_end(pi, s);
+  return KLEIN_OK;
+}
+
 static int stack_impl(const klein_model* m, const float* latents, const void* text, const float* refs,
                       float sigma, float sigma_next, const klein_seq* seq, float* v_out, const StackWs& w,
                       int n_img, int n_ref, int n_total, bool prepared, cudaStream_t s) {
   const klein_model_desc& d = m->d;
   const int B = seq->batch;
   const int n_txt = seq->n_txt;
+  int rc;
   if (!prepared) {
     if (launch_positions(w.pos, n_txt, seq->img_h, seq->img_w, seq->n_refs, seq->ref_h, seq->ref_w, s) ||
         launch_rope_table(w.pos, w.rope, n_total, 10000.f, s))
       return cuda_fail("positions / rope table");
+    if (d.txt_in && (rc = project_text(m, text, seq, w, s))) return rc;
   }
   // a2: timestep embedding + modulation
   int pi = prof_begin(kProfTimeMod, s);
-  int rc = klein_op_time_mod(m, sigma, sigma_next, n_ref > 0, w.mod, w.fmod, w.tscratch, 8 * kDim * sizeof(float),
-                             s);
+  rc = klein_op_time_mod(m, sigma, sigma_next, n_ref > 0, w.mod, w.fmod, w.tscratch, 8 * kDim * sizeof(float), s);
   if (rc) return rc;
   prof_end(pi, s);
   // a3: assemble [text | image | reference] rows of x
   pi = prof_begin(kProfOther, s);
-  if (launch_rows_to_f32(static_cast<const __nv_bfloat16*>(text), n_txt, w.x, n_total, 0, B, n_txt, s))
+  if (d.txt_in) {
+    for (int b = 0; b < B; ++b)
+      if (cudaMemcpyAsync(w.x + (size_t)b * n_total * kDim, w.txt + (size_t)b * n_txt * kDim,
+                          (size_t)n_txt * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return cuda_fail("text rows");
+  } else if (launch_rows_to_f32(static_cast<const __nv_bfloat16*>(text), n_txt, w.x, n_total, 0, B, n_txt, s)) {
     return cuda_fail("text rows");
+  }
   prof_end(pi, s);
   auto project = [&](const float* lat, int rows, const void* wproj, int row0) -> int {
     const int pc = prof_begin(kProfProj, s);
@@ -679,6 +716,11 @@ int klein_denoise(const klein_model* m, float* latents, const void* text, const 
     return cuda_fail("positions / rope table");
   }
   prof_end(pi, s);
+  // the text does not change across steps: project it once
+  if (m->d.txt_in && (rc = project_text(m, text, seq, w, s))) {
+    delete[] sig;
+    return rc;
+  }
   for (int i = 0; i < steps && rc == KLEIN_OK; ++i) {
     rc = stack_impl(m, latents, text, refs, sig[i], distilled ? sig[i + 1] : 0.f, seq, w.v, w, ni, nr, nt, true, s);
     if (rc) break;

@@ -358,11 +358,17 @@ def transformer(model, latents: np.ndarray, text: np.ndarray, ref_lat: np.ndarra
     through the output layer.
 
     model: klein_inputs.ModelWeights. latents [n_img, 128] (shared by the
-    batch), text [B, n_txt, DIM], ref_lat [n_ref, 128] or None.
+    batch), text [B, n_txt, DIM] or, when the model has the text input
+    projection, the stacked encoder hidden states [B, n_txt, 8 * 2560]
+    ([blog] / [guide] "The text encoder": hidden states of eight encoder
+    layers are stacked per token and projected linearly to the model width),
+    ref_lat [n_ref, 128] or None.
     If stage1_out is a dict, the stage-1 outputs per stream are stored in it.
     """
     misc = model.misc
     text = np.asarray(text, F64)
+    if "txt_in" in misc:
+        text = text @ np.asarray(misc["txt_in"], F64).T
     B, n_txt, _ = text.shape
     n_img = latents.shape[0]
     n_ref = 0 if ref_lat is None else ref_lat.shape[0]

@@ -167,3 +167,25 @@ def test_full_depth_denoise_matches_stored_oracle(kb):
     assert np.all(np.isfinite(got))
     assert cosine(got, ref) >= 0.999, cosine(got, ref)
     assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)
+
+
+def test_stack_forward_with_text_projection(kb):
+    # text given as the stacked encoder hidden states (8 x 2560 per token),
+    # projected to 3072 by the model's txt_in; batch 2 (distinct texts)
+    m = ki.ModelWeights(seed=0, distilled=True, n_stage1=1, n_joint=1, txt_in=True)
+    t = upload_model(m, with_ref=False)
+    model = kb.KleinModel(t)
+    n_txt, img = 24, (4, 5)
+    seq = kb.make_seq(2, n_txt, img[0], img[1])
+    n_img, _, _ = kb.klein_seq_tokens(seq)
+    lat = ki.noise_latents(2, n_img)
+    hid = ki.text_hidden_states(1, 2, n_txt)
+    v = torch.full((2, n_img, 128), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_stack_forward(model, to_f32(lat), to_bf16(hid), None, 0.6, 0.4, seq, v, ws)
+    torch.cuda.synchronize()
+    ref = o.transformer(m, lat, hid, None, o.positions(n_txt, img), 0.6, 0.4)
+    got = host(v)
+    assert np.all(np.isfinite(got))
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)

@@ -88,6 +88,19 @@ def test_generated_weights_match_parameter_layout():
         n += sum(a.size for a in m.stage1(mode)[0].values())
     n += sum(a.size for a in m.joint()[0].values())
     assert n == o.parameter_count(True, 1, 1, txt_in=False)
+    # with the 20480 -> 3072 text input projection
+    mt = ki.ModelWeights(seed=0, distilled=False, n_stage1=1, n_joint=1, txt_in=True)
+    n_t = sum(a.size for a in mt.misc.values())
+    assert n_t - sum(a.size for a in ki.misc_weights(0, False).values()) == 8 * 2560 * o.DIM
+    assert o.parameter_count(False, 1, 1, txt_in=True) - o.parameter_count(False, 1, 1, txt_in=False) == 8 * 2560 * o.DIM
+
+
+def test_text_projection_shapes(golden):
+    # eight 2560-wide encoder layers stack to the printed 20480, projected to the width
+    g = golden("structure.txt")
+    m = ki.ModelWeights(seed=0, distilled=False, n_stage1=1, n_joint=1, txt_in=True)
+    assert m.misc["txt_in"].shape == (g["dim"], g["text_stack_dim"])
+    assert ki.text_hidden_states(1, 2, 3).shape == (2, 3, g["text_stack_dim"])
 
 
 # ------------------------------------------------------- embeddings
