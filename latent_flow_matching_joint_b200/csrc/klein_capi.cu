@@ -270,6 +270,8 @@ struct StackWs {
   __nv_bfloat16* lat_bf;  // [max(n_img, n_ref)][128]
   float* v;          // [batch][n_img][128]
   float* txt;        // [batch][n_txt][3072] projected text (models with txt_in)
+  float* s1_txt;     // [batch][n_txt][3072] stage-1 output of the text stream (base model cache)
+  float* s1_ref;     // [n_ref][3072] stage-1 output of the reference stream (base model cache)
   BlockWs blk;
   size_t bytes;
 };
@@ -291,6 +293,8 @@ static StackWs carve_stack(void* base, int batch, int n_total, int n_img, int n_
   w.lat_bf = reinterpret_cast<__nv_bfloat16*>(take((size_t)(n_img > n_ref ? n_img : n_ref) * kLatent * 2));
   w.v = reinterpret_cast<float*>(take((size_t)batch * n_img * kLatent * sizeof(float)));
   w.txt = reinterpret_cast<float*>(take((size_t)batch * (n_total - n_img - n_ref) * kDim * sizeof(float)));
+  w.s1_txt = reinterpret_cast<float*>(take((size_t)batch * (n_total - n_img - n_ref) * kDim * sizeof(float)));
+  w.s1_ref = reinterpret_cast<float*>(take((size_t)n_ref * kDim * sizeof(float)));
   w.blk = carve_block(base ? static_cast<char*>(base) + off : nullptr, batch, n_total);
   off += w.blk.bytes;
   w.bytes = off;
@@ -552,12 +556,25 @@ static int project_text(const klein_model* m, const void* text, const klein_seq*
   return KLEIN_OK;
 }
 
+// Stage-1 cache of the text and reference streams. Their stage-1 output does
+// not depend on the noise level when the model has no target-level embedder
+// (base model: those streams are always modulated at t = 0), so a denoise
+// computes it at the first step and reuses it afterwards.
+enum StageOneCache { kCacheNone = 0, kCacheStore = 1, kCacheLoad = 2 };
+
+static int copy_rows_f32(float* dst, const float* src, size_t rows, cudaStream_t s) {
+  return cudaMemcpyAsync(dst, src, rows * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s) == cudaSuccess
+             ? KLEIN_OK
+             : cuda_fail("stage-1 cache copy");
+}
+
 static int stack_impl(const klein_model* m, const float* latents, const void* text, const float* refs,
                       float sigma, float sigma_next, const klein_seq* seq, float* v_out, const StackWs& w,
-                      int n_img, int n_ref, int n_total, bool prepared, cudaStream_t s) {
+                      int n_img, int n_ref, int n_total, bool prepared, int cache, cudaStream_t s) {
   const klein_model_desc& d = m->d;
   const int B = seq->batch;
   const int n_txt = seq->n_txt;
+  const bool load = cache == kCacheLoad;
   int rc;
   if (!prepared) {
     if (launch_positions(w.pos, n_txt, seq->img_h, seq->img_w, seq->n_refs, seq->ref_h, seq->ref_w, s) ||
@@ -572,7 +589,12 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
   prof_end(pi, s);
   // a3: assemble [text | image | reference] rows of x
   pi = prof_begin(kProfOther, s);
-  if (d.txt_in) {
+  if (load) {
+    for (int b = 0; b < B; ++b)
+      if ((rc = copy_rows_f32(w.x + (size_t)b * n_total * kDim, w.s1_txt + (size_t)b * n_txt * kDim, n_txt, s)))
+        return rc;
+    if (n_ref && (rc = copy_rows_f32(w.x + (size_t)(n_txt + n_img) * kDim, w.s1_ref, n_ref, s))) return rc;
+  } else if (d.txt_in) {
     for (int b = 0; b < B; ++b)
       if (cudaMemcpyAsync(w.x + (size_t)b * n_total * kDim, w.txt + (size_t)b * n_txt * kDim,
                           (size_t)n_txt * kDim * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -606,7 +628,7 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
     return KLEIN_OK;
   };
   if ((rc = project(latents, n_img, d.img_in, n_txt))) return rc;
-  if (n_ref && (rc = project(refs, n_ref, d.ref_in, n_txt + n_img))) return rc;
+  if (n_ref && !load && (rc = project(refs, n_ref, d.ref_in, n_txt + n_img))) return rc;
   // a8 stage 1: each stream through its own blocks, attending to itself.
   // The image and reference streams start from the same latents in every
   // batch item (the batch only varies the text, e.g. guidance's cond and
@@ -615,13 +637,19 @@ static int stack_impl(const klein_model* m, const float* latents, const void* te
   const int lo[3] = {0, n_txt, n_txt + n_img};
   const int cnt[3] = {n_txt, n_img, n_ref};
   for (int md = 0; md < 3; ++md) {
-    if (cnt[md] == 0) continue;
+    if (cnt[md] == 0 || (load && md != 1)) continue;
     const int nb = md == 0 ? B : 1;
     for (int i = 0; i < d.n_stage1; ++i) {
       rc = block_impl(&d.stage1[md][i], w.x, nb, n_total, lo[md], cnt[md], n_txt, n_img,
                       w.rope + (size_t)lo[md] * kPairs, w.mod, w.blk, s);
       if (rc) return rc;
     }
+  }
+  if (cache == kCacheStore) {
+    for (int b = 0; b < B; ++b)
+      if ((rc = copy_rows_f32(w.s1_txt + (size_t)b * n_txt * kDim, w.x + (size_t)b * n_total * kDim, n_txt, s)))
+        return rc;
+    if (n_ref && (rc = copy_rows_f32(w.s1_ref, w.x + (size_t)(n_txt + n_img) * kDim, n_ref, s))) return rc;
   }
   if (d.n_stage1 > 0) {
     for (int b = 1; b < B; ++b) {
@@ -684,7 +712,7 @@ int klein_stack_forward(const klein_model* m, const float* latents, const void* 
   if (rc) return rc;
   if (!v_out || !aligned16(v_out)) return fail(KLEIN_ERR_ALIGN, "v_out must be a 16-byte aligned device pointer");
   const StackWs w = carve_stack(ws, seq->batch, nt, ni, nr);
-  return stack_impl(m, latents, text, refs, sigma, sigma_next, seq, v_out, w, ni, nr, nt, false,
+  return stack_impl(m, latents, text, refs, sigma, sigma_next, seq, v_out, w, ni, nr, nt, false, kCacheNone,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -722,7 +750,10 @@ int klein_denoise(const klein_model* m, float* latents, const void* text, const 
     return rc;
   }
   for (int i = 0; i < steps && rc == KLEIN_OK; ++i) {
-    rc = stack_impl(m, latents, text, refs, sig[i], distilled ? sig[i + 1] : 0.f, seq, w.v, w, ni, nr, nt, true, s);
+    // base model: the text and reference streams' stage 1 is computed once
+    const int cache = distilled ? kCacheNone : (i == 0 ? kCacheStore : kCacheLoad);
+    rc = stack_impl(m, latents, text, refs, sig[i], distilled ? sig[i + 1] : 0.f, seq, w.v, w, ni, nr, nt, true, cache,
+                    s);
     if (rc) break;
     const float dsig = static_cast<float>(static_cast<double>(sig[i + 1]) - static_cast<double>(sig[i]));
     const int pi = prof_begin(kProfEuler, s);

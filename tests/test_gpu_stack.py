@@ -189,3 +189,21 @@ def test_stack_forward_with_text_projection(kb):
     assert np.all(np.isfinite(got))
     assert cosine(got, ref) >= 0.999, cosine(got, ref)
     assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)
+
+
+def test_denoise_base_with_reference_uses_stage1_cache(kb):
+    # base model (no target-level embedder): the text and reference streams'
+    # stage-1 output is computed at the first step and reused; the result
+    # must still match the oracle, which recomputes everything every step
+    m = ki.ModelWeights(seed=3, distilled=False, n_stage1=2, n_joint=1)
+    t = upload_model(m)
+    model = kb.KleinModel(t)
+    refs = ((3, 4),)
+    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 1, 20, 5, 4, refs, "cache")
+    x = to_f32(lat)
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 1.0, seq, ws)
+    torch.cuda.synchronize()
+    ref = o.denoise(m, lat, text, rl, o.positions(20, (5, 4), refs), 3)
+    assert cosine(host(x), ref) >= 0.999
+    assert max_err_ratio(host(x), ref) <= 5e-2
