@@ -199,11 +199,11 @@ def test_denoise_base_with_reference_uses_stage1_cache(kb):
     t = upload_model(m)
     model = kb.KleinModel(t)
     refs = ((3, 4),)
-    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 1, 20, 5, 4, refs, "cache")
+    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 2, 20, 5, 4, refs, "cache")
     x = to_f32(lat)
     ws = workspace(kb.klein_stack_workspace_size(seq))
-    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 1.0, seq, ws)
+    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 2.0, seq, ws)
     torch.cuda.synchronize()
-    ref = o.denoise(m, lat, text, rl, o.positions(20, (5, 4), refs), 3)
+    ref = o.denoise(m, lat, text, rl, o.positions(20, (5, 4), refs), 3, cfg=2.0)
     assert cosine(host(x), ref) >= 0.999
     assert max_err_ratio(host(x), ref) <= 5e-2
