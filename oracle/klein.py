@@ -34,6 +34,9 @@ import math
 
 import numpy as np
 
+from .fp8 import dequantize as fp8_dequantize
+from .fp8 import fake_quant as fp8_fake_quant
+
 DIM = 3072
 HEADS = 24
 HEAD_DIM = 128
@@ -307,26 +310,42 @@ def block(x: np.ndarray, pos: np.ndarray, mode_of_row: np.ndarray, mod: np.ndarr
     and added to x.
     If `rows` is given, only those output rows are computed (all rows still
     supply keys and values); the result is [B, len(rows), DIM].
+
+    Rowwise FP8 weights (keys w_in_q/w_in_s/w_out_q/w_out_s, from
+    oracle.fp8.quantize_block_weights): the weights are dequantised, and the
+    two GEMM inputs, the normalised rows h and the concatenated
+    [attention heads | SwiGLU hidden] rows, are quantised rowwise to e4m3
+    and dequantised before their GEMM (oracle.fp8 states the reading).
     """
     x = np.asarray(x, F64)
     B, R, _ = x.shape
     if rows is None:
         rows = np.arange(R)
     rows = np.asarray(rows)
+    fp8 = "w_in_q" in w
     h = modln(x, mode_of_row, mod)
-    w_q, w_k, w_v, w_g, w_u = _split_w_in(w["w_in"])
-    w_out = np.asarray(w["w_out"], F64)
-    w_o, w_d = w_out[:, :DIM], w_out[:, DIM:]
+    if fp8:
+        h = fp8_fake_quant(h)
+        w_in = fp8_dequantize(w["w_in_q"], w["w_in_s"])
+        w_out = fp8_dequantize(w["w_out_q"], w["w_out_s"])
+    else:
+        w_in = w["w_in"]
+        w_out = np.asarray(w["w_out"], F64)
+    w_q, w_k, w_v, w_g, w_u = _split_w_in(w_in)
     hr = h[:, rows]
     q = (hr @ w_q.T).reshape(B, len(rows), HEADS, HEAD_DIM)
     k = (h @ w_k.T).reshape(B, R, HEADS, HEAD_DIM)
     v = (h @ w_v.T).reshape(B, R, HEADS, HEAD_DIM)
     q = rope(rms_norm(q, w["q_norm"]), pos[rows])
     k = rope(rms_norm(k, w["k_norm"]), pos)
-    attn = attention(q, k, v).reshape(B, len(rows), DIM) @ w_o.T
-    mlp = swiglu(hr @ w_g.T, hr @ w_u.T) @ w_d.T
+    heads = attention(q, k, v).reshape(B, len(rows), DIM)
+    hidden = swiglu(hr @ w_g.T, hr @ w_u.T)
+    a_cat = np.concatenate([heads, hidden], axis=-1)
+    if fp8:
+        a_cat = fp8_fake_quant(a_cat)
+    out = a_cat @ w_out.T          # attention output projection + MLP down-projection
     gate = mod[mode_of_row[rows], 2]
-    return x[:, rows] + gate * (attn + mlp)
+    return x[:, rows] + gate * out
 
 
 def output_layer(x_img: np.ndarray, final_mod: np.ndarray, w_final: np.ndarray) -> np.ndarray:
