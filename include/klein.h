@@ -92,14 +92,15 @@ int klein_wait_probe(unsigned long long limit_ns, void* stream);
  *   0 modulated LayerNorm, 1 in-projection GEMM (QKV + MLP-in, fused
  *   epilogue), 2 attention, 3 out-projection GEMM (gated residual),
  *   4 timestep embedding + modulation, 5 input / output projections,
- *   6 Euler update, 7 other.
+ *   6 Euler update, 7 other, 8 rowwise e4m3 quantisation of the
+ *   out-projection's input (FP8 blocks only).
  * klein_profile_begin(max_launches) creates the events (host-side
  * resources; no device memory); klein_profile_end synchronises, writes the
  * summed milliseconds and launch counts per kind (arrays of
  * KLEIN_PROF_KINDS, either may be NULL) and releases the events. Returns
  * KLEIN_ERR_WORKSPACE if more launches happened than max_launches (those
  * were not timed). Not thread-safe; one profile at a time. */
-#define KLEIN_PROF_KINDS 8
+#define KLEIN_PROF_KINDS 9
 int klein_profile_begin(int max_launches);
 int klein_profile_end(double* ms, int* launches);
 
@@ -143,13 +144,37 @@ int klein_positions(const klein_seq* seq, float* pos, void* stream);
  *          gate(9216) | up(9216); the SwiGLU hidden is silu(gate) * up.
  *   w_out  bf16 [3072][12288]: input columns attention (3072, the attention
  *          output projection) | MLP down (9216).
- *   q_norm, k_norm  float [128]: QK-RMSNorm weights shared by all heads. */
+ *   q_norm, k_norm  float [128]: QK-RMSNorm weights shared by all heads.
+ *   w_in_scale, w_out_scale  NULL for a bf16 block. Both set: the block is
+ *          rowwise FP8 (the transformer's "fp8r" file, Diffusers release
+ *          blog, "Smaller GPUs, single files, and custom LoRA training"):
+ *          w_in and w_out then hold e4m3 codes (one byte per element, same
+ *          shapes) and w_in_scale float [27648], w_out_scale float [3072]
+ *          one scale per output row, as klein_quantize_rowwise_e4m3 writes
+ *          them. The block quantises its two GEMM inputs (the modulated
+ *          LayerNorm rows, and the [attention | SwiGLU] rows) the same way
+ *          per token and runs both GEMMs on e4m3 tensor cores with fp32
+ *          accumulation; everything else is as in the bf16 block. */
 typedef struct {
   const void* w_in;
   const void* w_out;
   const float* q_norm;
   const float* k_norm;
+  const float* w_in_scale;
+  const float* w_out_scale;
 } klein_block_weights;
+
+/* Rowwise e4m3 quantisation of a bf16 matrix src [rows][cols] (row pitch
+ * cols): codes [rows][cols] bytes, scale [rows] float. Per row, in fp32:
+ * amax = max |x|, inv = 448 / amax and scale = amax / 448 (correctly rounded
+ * divisions), code = e4m3(x * inv) rounded to nearest even and saturated to
+ * +-448 (OCP 8-bit floating point, E4M3: bias 7, no infinities); an all-zero
+ * row gets scale 0 and codes 0. This is how FP8 block weights are made
+ * (klein_block_weights). cols a multiple of 8, at most 12288; pointers
+ * 16-byte aligned; codes must not overlap src. Errors: KLEIN_ERR_SHAPE,
+ * KLEIN_ERR_ALIGN, KLEIN_ERR_INVALID_ARG. */
+int klein_quantize_rowwise_e4m3(const void* src, long long rows, int cols, void* codes, float* scale,
+                                void* stream);
 
 /* Workspace bytes for klein_block_forward on `rows` rows of `batch` items. */
 size_t klein_block_workspace_size(int batch, int rows);
@@ -286,6 +311,19 @@ int klein_op_euler(float* x, const float* v_cond, const float* v_uncond, long lo
 /* C[M][N] (float) = A[M][K] * B[N][K]^T, bf16 operands, tcgen05 tensor cores.
  * M >= 1, N a multiple of 128, K a multiple of 64. */
 int klein_op_gemm(const void* a, const void* b, float* c, int m, int n, int k, void* stream);
+
+/* C[m][n] (float) = a_scale[m] * b_scale[n] * sum_k A[m][k] * B[n][k], A and
+ * B e4m3 codes (bytes, row pitch K), on the e4m3 tensor-core GEMM of the FP8
+ * block. M >= 1, N a multiple of 256, K a multiple of 128. */
+int klein_op_gemm_e4m3(const void* a, const float* a_scale, const void* b, const float* b_scale, float* c, int m,
+                       int n, int k, void* stream);
+
+/* klein_op_modln with the output quantised rowwise to e4m3, as the FP8
+ * block's first step does: codes [batch][rows][3072] bytes, scale
+ * [batch][rows] float (the rule of klein_quantize_rowwise_e4m3, applied to
+ * the fp32 normalised rows). Per-stream modes as in klein_block_forward. */
+int klein_op_modln_e4m3(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
+                        const float* mod, long long mod_stride, void* codes, float* scale, void* stream);
 
 /* Softmax attention per (batch, head) over `rows` rows, scale 1/sqrt(128),
  * no mask. q, k: bf16 [batch][24][rows_pad][128]; vt: bf16

@@ -48,7 +48,8 @@ class KleinSeq(Structure):
 
 
 class KleinBlockWeights(Structure):
-    _fields_ = [("w_in", c_void_p), ("w_out", c_void_p), ("q_norm", c_void_p), ("k_norm", c_void_p)]
+    _fields_ = [("w_in", c_void_p), ("w_out", c_void_p), ("q_norm", c_void_p), ("k_norm", c_void_p),
+                ("w_in_scale", c_void_p), ("w_out_scale", c_void_p)]
 
 
 class KleinModelDesc(Structure):
@@ -90,6 +91,11 @@ _SIGS = {
     "klein_op_euler": (c_int, [c_void_p, c_void_p, c_void_p, c_longlong, c_float, c_float, c_void_p, c_float,
                                c_void_p]),
     "klein_op_gemm": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "klein_op_gemm_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                   c_void_p]),
+    "klein_op_modln_e4m3": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_longlong,
+                                    c_void_p, c_void_p, c_void_p]),
+    "klein_quantize_rowwise_e4m3": (c_int, [c_void_p, c_longlong, c_int, c_void_p, c_void_p, c_void_p]),
     "klein_op_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_longlong,
                                    c_void_p]),
     "klein_op_time_mod": (c_int, [c_void_p, c_float, c_float, c_int, c_void_p, c_void_p, c_void_p, c_size_t,
@@ -169,7 +175,7 @@ def klein_wait_probe(limit_ns: int, stream=None):
     _check(lib.klein_wait_probe(limit_ns, _stream(stream)))
 
 
-PROF_KINDS = ("modln", "gemm_in", "attention", "gemm_out", "time_mod", "projections", "euler", "other")
+PROF_KINDS = ("modln", "gemm_in", "attention", "gemm_out", "time_mod", "projections", "euler", "other", "quant")
 
 
 def klein_profile_begin(max_launches: int):
@@ -199,9 +205,32 @@ def klein_positions(seq: KleinSeq, pos, stream=None):
 
 
 def block_weights(w: dict) -> KleinBlockWeights:
-    """KleinBlockWeights from a dict of CUDA tensors w_in, w_out, q_norm, k_norm."""
+    """KleinBlockWeights from a dict of CUDA tensors w_in, w_out, q_norm, k_norm
+    (+ w_in_scale, w_out_scale for a rowwise FP8 block, see quantize_block_e4m3)."""
+    si, so = w.get("w_in_scale"), w.get("w_out_scale")
     return KleinBlockWeights(w["w_in"].data_ptr(), w["w_out"].data_ptr(), w["q_norm"].data_ptr(),
-                             w["k_norm"].data_ptr())
+                             w["k_norm"].data_ptr(), si.data_ptr() if si is not None else None,
+                             so.data_ptr() if so is not None else None)
+
+
+def klein_quantize_rowwise_e4m3(src, codes, scale, stream=None):
+    """Rowwise e4m3 codes (uint8, same shape) and scales (float32 [rows]) of a
+    bf16 [rows, cols] CUDA tensor."""
+    rows, cols = src.shape
+    _check(lib.klein_quantize_rowwise_e4m3(_ptr(src), rows, cols, _ptr(codes), _ptr(scale), _stream(stream)))
+
+
+def quantize_block_e4m3(w: dict, stream=None) -> dict:
+    """A rowwise FP8 copy of one block's bf16 weights (new device tensors)."""
+    import torch
+    out = {"q_norm": w["q_norm"], "k_norm": w["k_norm"]}
+    for name in ("w_in", "w_out"):
+        src = w[name]
+        codes = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+        scale = torch.empty(src.shape[0], dtype=torch.float32, device=src.device)
+        klein_quantize_rowwise_e4m3(src, codes, scale, stream)
+        out[name], out[name + "_scale"] = codes, scale
+    return out
 
 
 def klein_block_forward(w: dict, x, n_txt: int, n_img: int, pos, mod, ws, row0: int = 0, rows: int | None = None,
@@ -312,6 +341,20 @@ def klein_op_gemm(a, b, c, stream=None):
     m, k = a.shape
     n = b.shape[0]
     _check(lib.klein_op_gemm(_ptr(a), _ptr(b), _ptr(c), m, n, k, _stream(stream)))
+
+
+def klein_op_gemm_e4m3(a, a_scale, b, b_scale, c, stream=None):
+    m, k = a.shape
+    n = b.shape[0]
+    _check(lib.klein_op_gemm_e4m3(_ptr(a), _ptr(a_scale), _ptr(b), _ptr(b_scale), _ptr(c), m, n, k,
+                                  _stream(stream)))
+
+
+def klein_op_modln_e4m3(x, row0: int, rows: int, n_txt: int, n_img: int, mod, codes, scale, stream=None):
+    batch, n_total = x.shape[0], x.shape[1]
+    stride = mod.shape[-2] * mod.shape[-1]
+    _check(lib.klein_op_modln_e4m3(_ptr(x), batch, n_total, row0, rows, n_txt, n_img, _ptr(mod), stride,
+                                   _ptr(codes), _ptr(scale), _stream(stream)))
 
 
 def klein_op_attention(q, k, vt, rows: int, out, stream=None):

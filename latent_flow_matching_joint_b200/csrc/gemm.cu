@@ -1,5 +1,8 @@
 // Persistent tcgen05 GEMM, C = A * B^T, bf16 operands, fp32 accumulation in
-// tensor memory, fed by TMA, with the block's fused epilogues.
+// tensor memory, fed by TMA, with the block's fused epilogues. The CTA-pair
+// variant also runs rowwise-scaled e4m3 operands (kind::f8f6f4) for the FP8
+// block: same shared-memory bytes per stage (128 K elements instead of 64),
+// twice the MMA rate, and the two scales applied in the epilogue.
 //
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 per stage
@@ -43,14 +46,30 @@ __device__ __forceinline__ void store16(void* p, uint32_t a, uint32_t b, uint32_
 
 // ---- epilogues: one thread = one accumulator row; taddr = lane quarter base
 
-template <int BN>
+// e4m3 operands: the accumulator holds sum(code_a * code_b); the value is that
+// times the row's activation scale and the output channel's weight scale.
+__device__ __forceinline__ void dequant32(float* v, float sa, const float* sb) {
+  const float4* s4 = reinterpret_cast<const float4*>(sb);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = __ldg(s4 + i);
+    v[4 * i + 0] *= sa * t.x;
+    v[4 * i + 1] *= sa * t.y;
+    v[4 * i + 2] *= sa * t.z;
+    v[4 * i + 3] *= sa * t.w;
+  }
+}
+
+template <int BN, bool F8>
 __device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, bool f32) {
   const bool valid = r < g.rows;
+  const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   float v[32];
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     tmem_ld32(taddr + 32 * c, v);
     if (!valid) continue;
+    if (F8) dequant32(v, sa, g.b_scale + n_idx * BN + 32 * c);
     const int col = n_idx * BN + 32 * c;
     const int copies = g.replicate > 1 ? g.replicate : 1;
     for (int rep = 0; rep < copies; ++rep) {
@@ -71,8 +90,10 @@ __device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int
   }
 }
 
+template <bool F8>
 __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
   const bool valid = r < g.rows;
+  const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   float v[32];
   if (n_idx < g.b_split) {
     const int which = n_idx / 12;            // 0 q, 1 k, 2 v
@@ -82,11 +103,13 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
       const int head = head0 + hh;
       const uint32_t tcol = taddr + hh * 128;
       const long long bh = (long long)b * kHeads + head;
+      const float* sb = F8 ? g.b_scale + n_idx * 256 + hh * 128 : nullptr;
       if (which == 2) {
         __nv_bfloat16* dst = g.vt + bh * kHeadDim * g.rows_pad + r;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           tmem_ld32(tcol + 32 * c, v);
+          if (F8) dequant32(v, sa, sb + 32 * c);
           if (valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) dst[(long long)(32 * c + i) * g.rows_pad] = __float2bfloat16_rn(v[i]);
@@ -100,6 +123,7 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tcol + 32 * c, v);
+        if (F8) dequant32(v, sa, sb + 32 * c);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
       }
@@ -109,6 +133,7 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tcol + 32 * c, v);
         if (!valid) continue;
+        if (F8) dequant32(v, sa, sb + 32 * c);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -134,6 +159,10 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
       tmem_ld32(taddr + 32 * c, v);
       tmem_ld32(taddr + 128 + 32 * c, u);
       if (!valid) continue;
+      if (F8) {
+        dequant32(v, sa, g.b_scale + 3 * kDim + chunk * 128 + 32 * c);
+        dequant32(u, sa, g.b_scale + 3 * kDim + kMlp + chunk * 128 + 32 * c);
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16(silu(v[i]) * u[i], silu(v[i + 1]) * u[i + 1]);
@@ -146,9 +175,10 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
   }
 }
 
-template <int BN>
+template <int BN, bool F8>
 __device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
   const bool valid = r < g.rows;
+  const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   const int grow = g.x_row0 + r;
   const int mode = mode_of_row(grow, g.n_txt, g.n_img);
   const float* gate = g.mod + (long long)mode * 3 * kDim + 2 * kDim + n_idx * BN;
@@ -158,6 +188,7 @@ __device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int
   for (int c = 0; c < BN / 32; ++c) {
     tmem_ld32(taddr + 32 * c, v);
     if (!valid) continue;
+    if (F8) dequant32(v, sa, g.b_scale + n_idx * BN + 32 * c);
     float4* p = reinterpret_cast<float4*>(xr + 32 * c);
     const float4* gt = reinterpret_cast<const float4*>(gate + 32 * c);
 #pragma unroll
@@ -290,10 +321,10 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&acc_full[acc], acc_phase, 0x104)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (EPI == kEpiF32) epi_store<BN>(taddr, g, b, r, n_idx, true);
-      else if (EPI == kEpiBF16) epi_store<BN>(taddr, g, b, r, n_idx, false);
-      else if (EPI == kEpiQKV) epi_qkv(taddr, g, b, r, n_idx);
-      else epi_resid<BN>(taddr, g, b, r, n_idx);
+      if (EPI == kEpiF32) epi_store<BN, false>(taddr, g, b, r, n_idx, true);
+      else if (EPI == kEpiBF16) epi_store<BN, false>(taddr, g, b, r, n_idx, false);
+      else if (EPI == kEpiQKV) epi_qkv<false>(taddr, g, b, r, n_idx);
+      else epi_resid<BN, false>(taddr, g, b, r, n_idx);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -347,7 +378,7 @@ struct PairCfg {
   static constexpr int kThreads = 192;
 };
 
-template <int EPI>
+template <int EPI, bool F8>
 __global__ void __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const GemmArgs g) {
@@ -391,7 +422,8 @@ __global__ void __launch_bounds__(192, 1)
   const int total = m_tiles * g.n_tiles;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  constexpr uint32_t idesc = idesc_bf16_f32(256, 256);
+  constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(256, 256) : idesc_bf16_f32(256, 256);
+  constexpr int kBlockK = F8 ? 128 : 64;  // elements per 128-byte swizzle row
 
   if (warp == 0) {
     if (lane == 0) {
@@ -415,8 +447,8 @@ __global__ void __launch_bounds__(192, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStage);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* sa = smem + stage * Cfg::kStage;
-          tma_load_3d_pair(sa, &map_a, bar, kb * 64, row0, b);
-          tma_load_2d_pair(sa + Cfg::kStageA, &map_b, bar, kb * 64, brow);
+          tma_load_3d_pair(sa, &map_a, bar, kb * kBlockK, row0, b);
+          tma_load_2d_pair(sa + Cfg::kStageA, &map_b, bar, kb * kBlockK, brow);
           if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
@@ -440,8 +472,10 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t a0 = smem_u32(smem + stage * Cfg::kStage);
           const uint32_t b0 = a0 + Cfg::kStageA;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {
+            if (F8) umma_e4m3_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, (kb | k) != 0);
+            else umma_bf16_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, (kb | k) != 0);
+          }
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == Cfg::kStages) { stage = 0; phase ^= 1; }
         }
@@ -463,9 +497,9 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&acc_full[acc], acc_phase, 0x114)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (EPI == kEpiF32) epi_store<256>(taddr, g, b, r, n_idx, true);
-      else if (EPI == kEpiQKV) epi_qkv(taddr, g, b, r, n_idx);
-      else epi_resid<256>(taddr, g, b, r, n_idx);
+      if (EPI == kEpiF32) epi_store<256, F8>(taddr, g, b, r, n_idx, true);
+      else if (EPI == kEpiQKV) epi_qkv<F8>(taddr, g, b, r, n_idx);
+      else epi_resid<256, F8>(taddr, g, b, r, n_idx);
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
     }
@@ -481,7 +515,7 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
   using Cfg = PairCfg;
   static int max_pairs = 0;
@@ -497,28 +531,38 @@ static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const G
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs == 0) {
-    if (cudaFuncSetAttribute(gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+    if (cudaFuncSetAttribute(gemm_pair_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
         cudaSuccess)
       return -1;
     cfg.gridDim = dim3(2 * (num_sms() / 2));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<EPI>, &cfg) != cudaSuccess || n < 1) return -1;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<EPI, F8>, &cfg) != cudaSuccess || n < 1) return -1;
     max_pairs = n;
   }
   const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
   if (total <= 0) return 0;
   const int pairs = total < max_pairs ? total : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, ma, mb, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI, F8>, ma, mb, g);
   note_launch();
   return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
-int launch_gemm_pair(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
+int launch_gemm_pair(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s,
+                     int e4m3) {
+  if (e4m3) {
+    if (!g.a_scale || !g.b_scale) return -2;
+    switch (epi) {
+      case kEpiF32: return launch_pair_one<kEpiF32, true>(ma, mb, g, s);
+      case kEpiQKV: return launch_pair_one<kEpiQKV, true>(ma, mb, g, s);
+      case kEpiResid: return launch_pair_one<kEpiResid, true>(ma, mb, g, s);
+    }
+    return -2;
+  }
   switch (epi) {
-    case kEpiF32: return launch_pair_one<kEpiF32>(ma, mb, g, s);
-    case kEpiQKV: return launch_pair_one<kEpiQKV>(ma, mb, g, s);
-    case kEpiResid: return launch_pair_one<kEpiResid>(ma, mb, g, s);
+    case kEpiF32: return launch_pair_one<kEpiF32, false>(ma, mb, g, s);
+    case kEpiQKV: return launch_pair_one<kEpiQKV, false>(ma, mb, g, s);
+    case kEpiResid: return launch_pair_one<kEpiResid, false>(ma, mb, g, s);
   }
   return -2;
 }

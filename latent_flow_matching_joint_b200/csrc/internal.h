@@ -13,11 +13,12 @@ namespace klein {
 
 // 2-D bf16 tensor map over a row-major [outer][inner] matrix with row pitch
 // `row_bytes`; box = box_inner x box_outer elements, 128-byte swizzle.
+// bytes1 = 1: one-byte elements (e4m3 codes) instead of bf16.
 int make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                uint32_t box_inner, uint32_t box_outer);
+                uint32_t box_inner, uint32_t box_outer, int bytes1 = 0);
 // 3-D bf16 tensor map over [d2][d1][d0] with byte strides s1 (d1) and s2 (d2).
 int make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                uint64_t s2, uint32_t box0, uint32_t box1);
+                uint64_t s2, uint32_t box0, uint32_t box1, int bytes1 = 0);
 
 // ------------------------------------------------------------------ GEMM
 
@@ -57,13 +58,19 @@ struct GemmArgs {
   int x_row0;
   const float* mod;   // [3 modes][3][3072] (shift, scale, gate)
   int n_txt, n_img;
+  // e4m3 operands (launch_gemm_pair with e4m3 = 1): acc * a_scale[b * rows + r] * b_scale[B row]
+  const float* a_scale;
+  const float* b_scale;
 };
 
 // C[M,N] = A[M,K] * B[N,K]^T with epilogue `epi`; bn = 128 or 256.
 // Same product on CTA pairs (clusters of 2) with 256 x 256 tiles: args.m_tiles_per_b
 // counts 256-row tiles, args.n_tiles 256-column tiles; epi is kEpiF32, kEpiQKV or kEpiResid.
+// With e4m3 = 1 both operands are rowwise-scaled e4m3 codes (maps of bytes,
+// 128-byte boxes) and k_blocks counts 128-element K blocks; epi is kEpiQKV or
+// kEpiResid.
 int launch_gemm_pair(int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
-                     cudaStream_t stream);
+                     cudaStream_t stream, int e4m3 = 0);
 int launch_gemm(int bn, int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
                 cudaStream_t stream);
 
@@ -84,6 +91,17 @@ int launch_attention(const CUtensorMap& map_q, const CUtensorMap& map_k, const C
 int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16* h, int batch, int rows,
                  int n_txt, int n_img, const float* mod, long long mod_mode_stride, int single_mode,
                  cudaStream_t stream);
+// Same normalisation and modulation, output quantised rowwise to e4m3:
+// codes [batch][rows][3072] bytes and one fp32 scale per row ([batch][rows]).
+int launch_modln_e4m3(const float* x, long long x_bstride, int x_row0, uint8_t* codes, float* scale, int batch,
+                      int rows, int n_txt, int n_img, const float* mod, long long mod_mode_stride,
+                      cudaStream_t stream);
+// Rowwise e4m3 quantisation of bf16 rows: src row r at src + r * src_ld
+// (elements), codes of row r at dst + r * dst_ld (bytes), scale[r]. cols a
+// multiple of 8, at most 12288. dst may alias src when dst_ld >= cols and
+// dst_ld <= 2 * src_ld (each row is read whole before it is written).
+int launch_quantize_rows(const __nv_bfloat16* src, long long src_ld, uint8_t* dst, long long dst_ld, float* scale,
+                         long long rows, int cols, cudaStream_t stream);
 int launch_rope_table(const float* pos, float2* table, int rows, float theta, cudaStream_t stream);
 int launch_rope_apply(const __nv_bfloat16* in, __nv_bfloat16* out, const float2* table, int rows, int heads,
                       cudaStream_t stream);

@@ -74,6 +74,154 @@ int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16*
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
+// ---- rowwise e4m3 quantisation (the transformer's rowwise FP8 weights,
+// Diffusers release blog for FLUX.3 Image Klein, "Smaller GPUs, single files,
+// and custom LoRA training"). Decision in fp32: amax = max |x| over the row,
+// inv = 448 / amax and scale = amax / 448 (correctly rounded divisions),
+// code = e4m3_rn_satfinite(x * inv); an all-zero row has scale 0.
+
+__device__ __forceinline__ void e4m3_row_scales(float amax, float& inv, float& scale) {
+  inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+  scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
+}
+
+// modLN with the output quantised: one warp per row, as modln_kernel.
+__global__ void __launch_bounds__(256, 2) modln_e4m3_kernel(const float* __restrict__ x, long long x_bstride,
+                                                         int x_row0, uint32_t* __restrict__ codes,
+                                                         float* __restrict__ scale, int batch, int rows,
+                                                         int n_txt, int n_img, const float* __restrict__ mod,
+                                                         long long mod_stride) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= batch * rows) return;
+  const int b = warp / rows;
+  const int i = warp % rows;
+  const int grow = x_row0 + i;
+  const float4* src = reinterpret_cast<const float4*>(x + ((long long)b * x_bstride + grow) * kDim);
+  uint32_t* dst = codes + ((long long)b * rows + i) * (kDim / 4);
+  constexpr int kVec = kDim / 4 / 32;
+  float4 v[kVec];
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) v[t] = __ldg(src + lane + 32 * t);
+  float sum = 0.f;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) sum += (v[t].x + v[t].y) + (v[t].z + v[t].w);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum * (1.0f / kDim);
+  float sq = 0.f;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const float a = v[t].x - mean, bb = v[t].y - mean, c = v[t].z - mean, d = v[t].w - mean;
+    sq = fmaf(a, a, fmaf(bb, bb, fmaf(c, c, fmaf(d, d, sq))));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = rsqrtf(sq * (1.0f / kDim) + 1e-6f);
+  const int m = mode_of_row(grow, n_txt, n_img);
+  const float4* shift = reinterpret_cast<const float4*>(mod + m * mod_stride);
+  const float4* scl = reinterpret_cast<const float4*>(mod + m * mod_stride + kDim);
+  // The modulated rows are formed twice, identically: once for the row
+  // maximum and once for the codes, so that only x stays in registers.
+  float amax = 0.f;
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const int c4 = lane + 32 * t;
+    const float4 sc = __ldg(scl + c4);
+    const float4 sh = __ldg(shift + c4);
+    const float4 e = v[t];
+    const float h0 = fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x);
+    const float h1 = fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y);
+    const float h2 = fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z);
+    const float h3 = fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  float inv, s;
+  e4m3_row_scales(amax, inv, s);
+#pragma unroll
+  for (int t = 0; t < kVec; ++t) {
+    const int c4 = lane + 32 * t;
+    const float4 sc = __ldg(scl + c4);
+    const float4 sh = __ldg(shift + c4);
+    const float4 e = v[t];
+    const float h0 = fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x);
+    const float h1 = fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y);
+    const float h2 = fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z);
+    const float h3 = fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w);
+    dst[c4] = pack_e4m3x4(__fmul_rn(h0, inv), __fmul_rn(h1, inv), __fmul_rn(h2, inv), __fmul_rn(h3, inv));
+  }
+  if (lane == 0) scale[(long long)b * rows + i] = s;
+}
+
+int launch_modln_e4m3(const float* x, long long x_bstride, int x_row0, uint8_t* codes, float* scale, int batch,
+                      int rows, int n_txt, int n_img, const float* mod, long long mod_stride, cudaStream_t s) {
+  const long long warps = (long long)batch * rows;
+  if (warps <= 0) return 0;
+  const int blocks = (int)((warps + 7) / 8);
+  modln_e4m3_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, reinterpret_cast<uint32_t*>(codes), scale, batch,
+                                           rows, n_txt, n_img, mod, mod_stride);
+  note_launch();
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+}
+
+// One CTA of 256 threads per row; 8 bf16 per thread per chunk, at most 6
+// chunks (12288 columns). The whole row is in registers before the block-wide
+// max, so codes may overwrite the row's own source bytes.
+constexpr int kQuantMaxChunks = 6;
+
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* src, long long src_ld,
+                                                            uint8_t* dst, long long dst_ld,
+                                                            float* __restrict__ scale, int cols) {
+  __shared__ float red[8];
+  const long long row = blockIdx.x;
+  const int nchunks = cols >> 3;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + row * src_ld);
+  uint4 raw[kQuantMaxChunks];
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < kQuantMaxChunks; ++j) {
+    const int c = threadIdx.x + 256 * j;
+    raw[j] = c < nchunks ? s4[c] : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = unpack_bf16(w[q]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();  // every thread's loads of this row have returned
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  float inv, s;
+  e4m3_row_scales(amax, inv, s);
+  uint2* d2 = reinterpret_cast<uint2*>(dst + row * dst_ld);
+#pragma unroll
+  for (int j = 0; j < kQuantMaxChunks; ++j) {
+    const int c = threadIdx.x + 256 * j;
+    if (c >= nchunks) break;
+    const float2 f0 = unpack_bf16(raw[j].x), f1 = unpack_bf16(raw[j].y);
+    const float2 f2 = unpack_bf16(raw[j].z), f3 = unpack_bf16(raw[j].w);
+    d2[c] = make_uint2(pack_e4m3x4(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv), __fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv)),
+                       pack_e4m3x4(__fmul_rn(f2.x, inv), __fmul_rn(f2.y, inv), __fmul_rn(f3.x, inv), __fmul_rn(f3.y, inv)));
+  }
+  if (threadIdx.x == 0) scale[row] = s;
+}
+
+int launch_quantize_rows(const __nv_bfloat16* src, long long src_ld, uint8_t* dst, long long dst_ld, float* scale,
+                         long long rows, int cols, cudaStream_t s) {
+  if (rows <= 0) return 0;
+  if (cols <= 0 || cols % 8 || cols > 256 * 8 * kQuantMaxChunks || rows > 0x7fffffffLL) return -2;
+  quantize_rows_kernel<<<(unsigned)rows, 256, 0, s>>>(src, src_ld, dst, dst_ld, scale, cols);
+  note_launch();
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+}
+
 // bf16 rows -> fp32 rows of the residual stream: src [batch][rows][3072]
 // (batch stride src_bstride rows) into dst rows [dst_row0, dst_row0 + rows)
 // of each batch item (batch stride dst_bstride rows).

@@ -54,7 +54,7 @@ int num_sms() {
 // events are recorded then.
 
 enum ProfKind { kProfModln = 0, kProfGemmIn, kProfAttn, kProfGemmOut, kProfTimeMod, kProfProj, kProfEuler,
-                kProfOther, kProfKinds };
+                kProfOther, kProfQuant, kProfKinds };
 
 struct Profiler {
   bool on = false;
@@ -93,26 +93,28 @@ static int get_encode() {
 }
 
 int make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                uint32_t box_inner, uint32_t box_outer) {
+                uint32_t box_inner, uint32_t box_outer, int bytes1) {
   if (get_encode()) return -1;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  const CUtensorMapDataType dt = bytes1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
 int make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                uint64_t s2, uint32_t box0, uint32_t box1) {
+                uint64_t s2, uint32_t box0, uint32_t box1, int bytes1) {
   if (get_encode()) return -1;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {s1, s2};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  const CUtensorMapDataType dt = bytes1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
@@ -127,6 +129,7 @@ static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t
 struct BlockWs {
   __nv_bfloat16 *h, *q, *k, *vt, *a_out;
   float2* rope;
+  float *sa_h, *sa_o;  // FP8 blocks: per-row scales of the two GEMM inputs
   int rows_pad;
   size_t bytes;
 };
@@ -147,6 +150,8 @@ static BlockWs carve_block(void* base, int batch, int rows) {
   w.vt = reinterpret_cast<__nv_bfloat16*>(take((size_t)batch * kHeads * rp * kHeadDim * 2));
   w.a_out = reinterpret_cast<__nv_bfloat16*>(take((size_t)batch * rows * kOutK * 2));
   w.rope = reinterpret_cast<float2*>(take((size_t)rows * kPairs * sizeof(float2)));
+  w.sa_h = reinterpret_cast<float*>(take((size_t)batch * rows * sizeof(float)));
+  w.sa_o = reinterpret_cast<float*>(take((size_t)batch * rows * sizeof(float)));
   w.bytes = off;
   return w;
 }
@@ -171,30 +176,41 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
                       int n_txt, int n_img, const float2* rope, const float* mod, const BlockWs& w,
                       cudaStream_t s) {
   const int rp = round_up(rows, 128);
+  // Rowwise FP8 blocks: both GEMMs on e4m3 codes (CTA pairs); the GEMM
+  // inputs are quantised per row where they are made (modLN) or just before
+  // the out-projection (in place, over the bf16 [attention | SwiGLU] rows).
+  const bool f8 = wt->w_in_scale != nullptr;
+  const int rows_per_tile = f8 ? 256 : kGemmRowsPerTile;
   // a4: modulated LayerNorm
   int pi = prof_begin(kProfModln, s);
-  if (launch_modln(x, n_total, row0, w.h, batch, rows, n_txt, n_img, mod, 3 * kDim, 0, s))
-    return cuda_fail("modln launch");
+  const int mrc = f8 ? launch_modln_e4m3(x, n_total, row0, reinterpret_cast<uint8_t*>(w.h), w.sa_h, batch, rows,
+                                         n_txt, n_img, mod, 3 * kDim, s)
+                     : launch_modln(x, n_total, row0, w.h, batch, rows, n_txt, n_img, mod, 3 * kDim, 0, s);
+  if (mrc) return cuda_fail("modln launch");
   prof_end(pi, s);
   // a5: fused in-projection
   CUtensorMap m_h, m_win, m_q, m_k, m_vt, m_aout, m_wout;
-  if (make_map_3d(&m_h, w.h, kDim, rows, batch, (uint64_t)kDim * 2, (uint64_t)rows * kDim * 2, 64, 128) ||
-      make_map_2d(&m_win, wt->w_in, kDim, kInCols, (uint64_t)kDim * 2, 64, 128) ||
+  const int eb = f8 ? 1 : 2;                // operand bytes per element
+  const uint32_t bk = f8 ? 128 : 64;        // elements per 128-byte K box
+  if (make_map_3d(&m_h, w.h, kDim, rows, batch, (uint64_t)kDim * eb, (uint64_t)rows * kDim * eb, bk, 128, f8) ||
+      make_map_2d(&m_win, wt->w_in, kDim, kInCols, (uint64_t)kDim * eb, bk, 128, f8) ||
       make_map_3d(&m_q, w.q, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rp * kHeadDim * 2,
                   64, 128) ||
       make_map_3d(&m_k, w.k, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rp * kHeadDim * 2,
                   64, 128) ||
       make_map_3d(&m_vt, w.vt, rows, kHeadDim, (uint64_t)batch * kHeads, (uint64_t)rp * 2,
                   (uint64_t)rp * kHeadDim * 2, 64, 128) ||
-      make_map_3d(&m_aout, w.a_out, kOutK, rows, batch, (uint64_t)kOutK * 2, (uint64_t)rows * kOutK * 2, 64, 128) ||
-      make_map_2d(&m_wout, wt->w_out, kOutK, kDim, (uint64_t)kOutK * 2, 64, 128))
+      // the out-projection's A keeps the bf16 row pitch: FP8 codes are written in place
+      make_map_3d(&m_aout, w.a_out, kOutK, rows, batch, (uint64_t)kOutK * 2, (uint64_t)rows * kOutK * 2, bk, 128,
+                  f8) ||
+      make_map_2d(&m_wout, wt->w_out, kOutK, kDim, (uint64_t)kOutK * eb, bk, 128, f8))
     return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   GemmArgs g{};
   g.batch = batch;
   g.rows = rows;
-  g.m_tiles_per_b = (rows + kGemmRowsPerTile - 1) / kGemmRowsPerTile;
+  g.m_tiles_per_b = (rows + rows_per_tile - 1) / rows_per_tile;
   g.n_tiles = 36 + kMlp / 128;
-  g.k_blocks = kDim / 64;
+  g.k_blocks = kDim / static_cast<int>(bk);
   g.b_split = 36;
   g.q = w.q;
   g.k = w.k;
@@ -204,8 +220,11 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   g.k_norm = wt->k_norm;
   g.rope = rope;
   g.rows_pad = rp;
+  g.a_scale = w.sa_h;
+  g.b_scale = wt->w_in_scale;
   pi = prof_begin(kProfGemmIn, s);
-  if (launch_block_gemm(kEpiQKV, m_h, m_win, g, s)) return cuda_fail("in-projection GEMM launch");
+  if (f8 ? launch_gemm_pair(kEpiQKV, m_h, m_win, g, s, 1) : launch_block_gemm(kEpiQKV, m_h, m_win, g, s))
+    return cuda_fail("in-projection GEMM launch");
   prof_end(pi, s);
   // a6: attention
   AttnArgs at{};
@@ -219,13 +238,20 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   pi = prof_begin(kProfAttn, s);
   if (launch_attention(m_q, m_k, m_vt, at, s)) return cuda_fail("attention launch");
   prof_end(pi, s);
+  if (f8) {
+    pi = prof_begin(kProfQuant, s);
+    if (launch_quantize_rows(w.a_out, kOutK, reinterpret_cast<uint8_t*>(w.a_out), (long long)kOutK * 2, w.sa_o,
+                             (long long)batch * rows, kOutK, s))
+      return cuda_fail("quantisation launch");
+    prof_end(pi, s);
+  }
   // a7: out-projection + gated residual
   GemmArgs o{};
   o.batch = batch;
   o.rows = rows;
-  o.m_tiles_per_b = (rows + kGemmRowsPerTile - 1) / kGemmRowsPerTile;
+  o.m_tiles_per_b = (rows + rows_per_tile - 1) / rows_per_tile;
   o.n_tiles = kDim / 256;
-  o.k_blocks = kOutK / 64;
+  o.k_blocks = kOutK / static_cast<int>(bk);
   o.n_fastest = 1;
   o.x = x;
   o.x_bstride = n_total;
@@ -233,8 +259,11 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   o.mod = mod;
   o.n_txt = n_txt;
   o.n_img = n_img;
+  o.a_scale = w.sa_o;
+  o.b_scale = wt->w_out_scale;
   pi = prof_begin(kProfGemmOut, s);
-  if (launch_block_gemm(kEpiResid, m_aout, m_wout, o, s)) return cuda_fail("out-projection GEMM launch");
+  if (f8 ? launch_gemm_pair(kEpiResid, m_aout, m_wout, o, s, 1) : launch_block_gemm(kEpiResid, m_aout, m_wout, o, s))
+    return cuda_fail("out-projection GEMM launch");
   prof_end(pi, s);
   return KLEIN_OK;
 }
@@ -313,7 +342,7 @@ extern "C" {
 
 const char* klein_last_error(void) { return g_msg; }
 
-int klein_version(void) { return 101; }
+int klein_version(void) { return 102; }
 
 long long klein_launch_count(void) { return g_launches; }
 
@@ -444,6 +473,10 @@ static int check_block_weights(const klein_block_weights* w) {
     return fail(KLEIN_ERR_INVALID_ARG, "block weights incomplete");
   if (!aligned16(w->w_in) || !aligned16(w->w_out) || !aligned16(w->q_norm) || !aligned16(w->k_norm))
     return fail(KLEIN_ERR_ALIGN, "block weights must be 16-byte aligned");
+  if ((w->w_in_scale == nullptr) != (w->w_out_scale == nullptr))
+    return fail(KLEIN_ERR_INVALID_ARG, "FP8 block weights need both w_in_scale and w_out_scale");
+  if ((w->w_in_scale && !aligned16(w->w_in_scale)) || (w->w_out_scale && !aligned16(w->w_out_scale)))
+    return fail(KLEIN_ERR_ALIGN, "weight scales must be 16-byte aligned");
   return KLEIN_OK;
 }
 
@@ -832,6 +865,60 @@ int klein_op_gemm(const void* a, const void* b, float* c, int m, int n, int k, v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rc = wide ? launch_block_gemm(kEpiF32, ma, mb, g, s) : launch_gemm(128, kEpiF32, ma, mb, g, s);
   if (rc) return cuda_fail("gemm launch");
+  return KLEIN_OK;
+}
+
+int klein_op_gemm_e4m3(const void* a, const float* a_scale, const void* b, const float* b_scale, float* c, int m,
+                       int n, int k, void* stream) {
+  if (!a || !a_scale || !b || !b_scale || !c) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c) || !aligned16(a_scale) || !aligned16(b_scale))
+    return fail(KLEIN_ERR_ALIGN, "unaligned pointer");
+  if (m < 1 || n < 256 || (n % 256) != 0 || k < 128 || (k % 128) != 0)
+    return fail(KLEIN_ERR_SHAPE, "need M >= 1, N a multiple of 256, K a multiple of 128");
+  CUtensorMap ma, mb;
+  if (make_map_3d(&ma, a, k, m, 1, (uint64_t)k, (uint64_t)m * k, 128, 128, 1) ||
+      make_map_2d(&mb, b, k, n, (uint64_t)k, 128, 128, 1))
+    return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  GemmArgs g{};
+  g.batch = 1;
+  g.rows = m;
+  g.m_tiles_per_b = (m + 255) / 256;
+  g.n_tiles = n / 256;
+  g.k_blocks = k / 128;
+  g.out = c;
+  g.out_ld = n;
+  g.out_bstride = m;
+  g.a_scale = a_scale;
+  g.b_scale = b_scale;
+  if (launch_gemm_pair(kEpiF32, ma, mb, g, static_cast<cudaStream_t>(stream), 1)) return cuda_fail("gemm launch");
+  return KLEIN_OK;
+}
+
+int klein_quantize_rowwise_e4m3(const void* src, long long rows, int cols, void* codes, float* scale,
+                                void* stream) {
+  if (!src || !codes || !scale) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(src) || !aligned16(codes) || !aligned16(scale)) return fail(KLEIN_ERR_ALIGN, "unaligned pointer");
+  if (rows < 1 || rows > 0x7fffffffLL || cols < 8 || (cols % 8) != 0 || cols > kOutK)
+    return fail(KLEIN_ERR_SHAPE, "need rows >= 1 and cols a multiple of 8 in [8, 12288]");
+  const char* s0 = static_cast<const char*>(src);
+  const char* c0 = static_cast<const char*>(codes);
+  if (c0 < s0 + rows * cols * 2 && s0 < c0 + rows * cols)
+    return fail(KLEIN_ERR_INVALID_ARG, "codes overlap src");
+  if (launch_quantize_rows(static_cast<const __nv_bfloat16*>(src), cols, static_cast<uint8_t*>(codes), cols, scale,
+                           rows, cols, static_cast<cudaStream_t>(stream)))
+    return cuda_fail("quantisation launch");
+  return KLEIN_OK;
+}
+
+int klein_op_modln_e4m3(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
+                        const float* mod, long long mod_stride, void* codes, float* scale, void* stream) {
+  if (!x || !mod || !codes || !scale) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(x) || !aligned16(mod) || !aligned16(codes) || !aligned16(scale) || (mod_stride % 4) != 0)
+    return fail(KLEIN_ERR_ALIGN, "pointers must be 16-byte aligned, mod_stride a multiple of 4");
+  if (batch < 1 || rows < 1 || row0 < 0 || row0 + rows > n_total) return fail(KLEIN_ERR_SHAPE, "bad row range");
+  if (launch_modln_e4m3(static_cast<const float*>(x), n_total, row0, static_cast<uint8_t*>(codes), scale, batch,
+                        rows, n_txt, n_img, mod, mod_stride, static_cast<cudaStream_t>(stream)))
+    return cuda_fail("modln launch");
   return KLEIN_OK;
 }
 

@@ -13,10 +13,12 @@ namespace klein {
 // Largest batch * round_up(rows, 128) the fixed scratch can hold.
 constexpr int kStaticMaxRows = 256;
 // Bytes of carve_block(1, kStaticMaxRows): h, q, k, v^T, attention|SwiGLU
-// operand, RoPE table (every region is a multiple of 256 bytes).
+// operand, RoPE table, the two per-row FP8 scale vectors (every region is a
+// multiple of 256 bytes).
 constexpr size_t kStaticWsBytes = (size_t)kStaticMaxRows * kDim * 2 +
                                   3 * (size_t)kHeads * kStaticMaxRows * kHeadDim * 2 +
-                                  (size_t)kStaticMaxRows * kOutK * 2 + (size_t)kStaticMaxRows * kPairs * sizeof(float2);
+                                  (size_t)kStaticMaxRows * kOutK * 2 + (size_t)kStaticMaxRows * kPairs * sizeof(float2) +
+                                  2 * (size_t)kStaticMaxRows * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 
