@@ -125,6 +125,12 @@ def test_device_block_weights_match_oracle_codes(kb, fp8_weights):
         np.testing.assert_array_equal(wd[name + "_scale"].cpu().numpy(), wq[name + "_s"])
 
 
+# Worst-element bound of the FP8 block against the FP8 oracle, x RMS(output):
+# about 1.5 x the effect of one bf16 rounding of the out-projection input
+# ahead of its quantisation (0.083, pinned on the CPU in
+# tests/test_oracle_fp8.py).
+FP8_MAX_ERR = 0.12
+
 FP8_CASES = {
     "config1": dict(batch=1, n_txt=80, img=(8, 8), refs=(), view="joint"),
     "ragged_ref_b2": dict(batch=2, n_txt=77, img=(9, 7), refs=((3, 5),), view="joint"),
@@ -161,16 +167,17 @@ def test_fp8_block_matches_oracle(kb, fp8_weights, name):
     assert np.all(np.isfinite(g))
     d_got, d_ref = g - x[:, sl], ref - x[:, sl]
     # The GPU stores the [attention | SwiGLU] rows in bf16 before quantising
-    # them (the oracle quantises its float64 rows): a bf16 rounding (2^-9
-    # relative) moves about 2^-9 / 2^-4 ~ 3 % of those values across an e4m3
-    # rounding boundary, each by one code step (up to 2^-3 relative), which
-    # is ~1 % RMS of the block update; attention and GEMM rounding add the
-    # bf16 path's own ~0.5 %. Bound: 3 % RMS of the update, and a max error
-    # of 3e-2 x RMS(block output).
+    # them (the oracle quantises its float64 rows): a bf16 rounding moves a
+    # few per cent of those values across an e4m3 rounding boundary, each by
+    # one code step (up to 2^-3 relative). tests/test_oracle_fp8.py measures
+    # that effect on the oracle itself (FP8_STORAGE_*): about 1.3 % RMS of the
+    # block update and 8 % of RMS(output) at the worst element. Bounds: 3 %
+    # RMS of the update, cosine >= 0.999, and FP8_MAX_ERR x RMS(output) at the
+    # worst element.
     rel = rms(d_got - d_ref) / rms(d_ref)
     assert rel <= 3e-2, rel
     assert cosine(d_got, d_ref) >= 0.999
-    assert max_err_ratio(g, ref) <= 3e-2, max_err_ratio(g, ref)
+    assert max_err_ratio(g, ref) <= FP8_MAX_ERR, max_err_ratio(g, ref)
     # and the GPU computes the FP8 method, not the bf16 one: its distance to
     # the FP8 oracle is well below the FP8 oracle's distance to the exact block
     if name == "config1":
