@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "joint-block TFLOP/s & denoise steps/s at 1024² (frac of B200 BF16 peak)"
 DIM, MLP, LAT = 3072, 9216, 128
+DTYPES = {"bf16": "bf16", "fp8": "e4m3 rowwise (block GEMMs), bf16 elsewhere"}
 
 WORKLOADS = {
     # name: (batch, n_txt, img grid, refs, steps, cfg, distilled, description)
@@ -40,6 +41,10 @@ WORKLOADS = {
                 "base 2048x2048 denoise: 560 text + 128x128 image tokens (16944), 50 steps, CFG 3.5 as batch 2"),
 }
 
+
+# Rowwise FP8 (e4m3) runs the two block GEMMs at the e4m3 tensor rate: the
+# measured bf16 peak times the nominal dense ratio (4.5 / 2.25 PFLOP/s).
+FP8_OVER_BF16 = 2.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of the in-projection GEMM
 # (gemm_pair_kernel<2>), mean over the first 42 launches of a t2i denoise, from
@@ -82,23 +87,29 @@ def step_flops(batch, n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
     return batch * f
 
 
-def executed_step_flops(batch, n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
-    """FLOPs the library executes per denoiser call: the image and reference
-    streams' stage-1 blocks run once for the whole batch (their inputs are the
-    same in every batch item), the text stream per batch item."""
+def executed_denoise_flops(batch, n_txt, n_img, n_ref, steps, distilled, n_stage1=5, n_joint=28):
+    """FLOPs the library executes over one denoise of `steps` Euler steps: the
+    image and reference streams' stage-1 blocks run once for the whole batch
+    (their inputs are the same in every batch item), the text stream per
+    batch item; without the target-level embedder (base model) the text and
+    reference streams' stage 1 and the reference projection run at the
+    first step only (their t = 0 output is cached)."""
     n = n_txt + n_img + n_ref
+    ctx_steps = steps if distilled else 1
     f = 0.0
-    for r, nb in ((n_txt, batch), (n_img, 1), (n_ref, 1)):
+    for r, nb, k in ((n_txt, batch, ctx_steps), (n_img, 1, steps), (n_ref, 1, ctx_steps)):
         if r:
-            f += nb * n_stage1 * (r * block_gemm_flops_per_token() + attn_flops(r))
-    f += batch * n_joint * (n * block_gemm_flops_per_token() + attn_flops(n))
-    f += 2.0 * (n_img + n_ref) * LAT * DIM + batch * 2.0 * n_img * DIM * LAT
+            f += k * nb * n_stage1 * (r * block_gemm_flops_per_token() + attn_flops(r))
+    f += steps * batch * n_joint * (n * block_gemm_flops_per_token() + attn_flops(n))
+    f += steps * 2.0 * n_img * LAT * DIM + ctx_steps * 2.0 * n_ref * LAT * DIM + steps * batch * 2.0 * n_img * DIM * LAT
     return f
 
 
-def gemm_in_rows_per_step(batch, n_txt, n_img, n_ref, n_stage1=5, n_joint=28):
-    """Rows the in-projection GEMM processes per denoiser call (as executed)."""
-    return n_stage1 * (batch * n_txt + n_img + n_ref) + n_joint * batch * (n_txt + n_img + n_ref)
+def gemm_in_rows_per_denoise(batch, n_txt, n_img, n_ref, steps, distilled, n_stage1=5, n_joint=28):
+    """Rows the in-projection GEMM processes over one denoise (as executed)."""
+    ctx_steps = steps if distilled else 1
+    return (n_stage1 * (ctx_steps * (batch * n_txt + n_ref) + steps * n_img)
+            + steps * n_joint * batch * (n_txt + n_img + n_ref))
 
 
 # ------------------------------------------------------------------ ranks
@@ -258,6 +269,17 @@ def random_block(g, dev):
             "k_norm": 1.0 + 0.1 * torch.randn(128, generator=g, device=dev)}
 
 
+def to_precision(t, precision):
+    """Rowwise FP8 copies of every block of a model dict (the bf16 block
+    weights are dropped); other weights stay bf16."""
+    if precision != "fp8":
+        return t
+    import latent_flow_matching_joint_b200 as kb
+    t["stage1"] = {m: [kb.quantize_block_e4m3(b) for b in bl] for m, bl in t["stage1"].items()}
+    t["joint"] = [kb.quantize_block_e4m3(b) for b in t["joint"]]
+    return t
+
+
 def random_model(dev, distilled, with_ref, seed=0):
     import torch
     g = torch.Generator(device=dev).manual_seed(seed)
@@ -287,6 +309,8 @@ def run_block_only(args):
     torch.cuda.set_device(0)
     g = torch.Generator(device=dev).manual_seed(0)
     bw = random_block(g, dev)
+    if args.precision == "fp8":
+        bw = kb.quantize_block_e4m3(bw)
     x = torch.randn(1, 4608, DIM, generator=g, device=dev)
     pos = torch.empty(4608, 4, device=dev)
     kb.klein_positions(kb.make_seq(1, 512, 64, 64), pos)
@@ -310,8 +334,9 @@ def run_block_only(args):
         raise RuntimeError(msg)
     print(json.dumps({"metric": "joint-block TFLOP/s at 512+4096 tokens", "value": flops / (ms / 1e3) / 1e12,
                       "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
-                      "frac_of_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16"], "dtype": "bf16",
-                      "config": {"workload": "one joint block, 512 text + 64x64 image tokens, batch 1"}}), flush=True)
+                      "frac_of_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16"], "dtype": DTYPES[args.precision],
+                      "config": {"workload": "one joint block, 512 text + 64x64 image tokens, batch 1",
+                                 "precision": args.precision}}), flush=True)
     return 0
 
 
@@ -335,8 +360,9 @@ def run_ours(args):
     batch, n_txt, grid, refs, steps, cfg, distilled, desc = WORKLOADS[args.workload]
     seq = kb.make_seq(batch, n_txt, grid[0], grid[1], refs)
     n_img, n_ref, n_total = kb.klein_seq_tokens(seq)
-    model_t = random_model(dev, distilled, bool(refs), seed=0)
+    model_t = to_precision(random_model(dev, distilled, bool(refs), seed=0), args.precision)
     model = kb.KleinModel(model_t)
+    fp8 = args.precision == "fp8"
     g = torch.Generator(device=dev).manual_seed(1 + rank)
     noise = torch.randn(n_img, LAT, generator=g, device=dev)
     text = torch.randn(batch, n_txt, DIM, generator=g, device=dev).to(torch.bfloat16)
@@ -392,15 +418,18 @@ def run_ours(args):
     tot = sum(v[0] for v in prof.values())
     top = max(prof, key=lambda k: prof[k][0])
     gi_ms, gi_n = prof["gemm_in"]
-    gi_flops = gemm_in_rows_per_step(batch, n_txt, n_img, n_ref) * steps * args.steps * 2.0 * DIM * (3 * DIM + 2 * MLP)
+    gi_flops = gemm_in_rows_per_denoise(batch, n_txt, n_img, n_ref, steps, distilled) * args.steps * 2.0 * DIM * (
+        3 * DIM + 2 * MLP)
     gi_avg_ms = gi_ms / max(gi_n, 1)
     achieved = gi_flops / (gi_ms / 1e3) / 1e12 if gi_ms > 0 else 0.0
-    roofline = {"kernel": "gemm_in (fused QKV + MLP-in, tcgen05)", "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"],
-                "traffic": GEMM_IN_TRAFFIC_BYTES if args.workload == "t2i" else None,
+    gi_peak = peaks["bf16_sustained"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    roofline = {"kernel": "gemm_in (fused QKV + MLP-in, tcgen05" + (", e4m3)" if fp8 else ")"), "bound": "tensor",
+                "achieved": achieved, "peak": gi_peak, "unit": "TFLOP/s", "frac": achieved / gi_peak,
+                "traffic": GEMM_IN_TRAFFIC_BYTES if args.workload == "t2i" and not fp8 else None,
                 "traffic_unit": "bytes per launch (ncu dram read + write)",
                 "avg_launch_ms": gi_avg_ms, "launches": gi_n,
-                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
+                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"
+                + (" x 2 (nominal e4m3 / bf16 dense ratio)" if fp8 else "")}
 
     # ---- end to end through the public API with host buffers
     noise_h = noise.cpu().pin_memory()
@@ -462,16 +491,19 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "denoise steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_image, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": DTYPES[args.precision], "data": "synthetic",
         "config": {"workload": desc, "global_batch": world * batch, "seq_len": n_total, "parallelism": f"replicas x{world}",
                    "euler_steps_per_bench_step": steps, "cfg": cfg, "distilled": distilled,
-                   "l2": "working set > L2 (11 GB of weights streamed per Euler step)",
-                   "weights": "random init N(0, 1/fan_in), bf16", "inputs": "N(0,1) noise and text embeddings"},
+                   "precision": args.precision,
+                   "l2": "working set > L2 (" + ("5.6" if fp8 else "11") + " GB of weights streamed per Euler step)",
+                   "weights": "random init N(0, 1/fan_in), bf16" + (
+                       "; block weights rowwise e4m3 (one scale per output row)" if fp8 else ""),
+                   "inputs": "N(0,1) noise and text embeddings"},
         # the method's FLOPs per step (every batch item's streams counted)
         "tflops_per_gpu": f_step * steps * args.steps / (ms / 1e3) / 1e12,
         "denoise_frac_of_peak": f_step * steps * args.steps / (ms / 1e3) / 1e12 / peaks["bf16_sustained"],
         # the FLOPs actually executed (shared image / reference stage 1 under a batch)
-        "executed_tflops_per_gpu": executed_step_flops(batch, n_txt, n_img, n_ref) * steps * args.steps
+        "executed_tflops_per_gpu": executed_denoise_flops(batch, n_txt, n_img, n_ref, steps, distilled) * args.steps
         / (ms / 1e3) / 1e12,
         "roofline": roofline,
         "kernels": {k: {"ms": v[0], "launches": v[1], "share": (v[0] / tot if tot else 0.0)} for k, v in prof.items()},
@@ -501,6 +533,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=tuple(WORKLOADS) + ("block",), default="t2i")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--precision", choices=tuple(DTYPES), default="bf16",
+                    help="block GEMM operands: bf16, or rowwise FP8 (e4m3 codes, one scale per row)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
