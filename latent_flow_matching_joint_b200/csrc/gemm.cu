@@ -24,6 +24,10 @@
 #include "common.cuh"
 #include "internal.h"
 
+#ifndef KLEIN_PAIR_EPI_WARPS
+#define KLEIN_PAIR_EPI_WARPS 8
+#endif
+
 namespace klein {
 
 template <int BN>
@@ -60,13 +64,17 @@ __device__ __forceinline__ void dequant32(float* v, float sa, const float* sb) {
   }
 }
 
+// part / nparts: this warp's share of the tile's columns when several
+// epilogue warps serve the same TMEM lane quarter.
 template <int BN, bool F8>
-__device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, bool f32) {
+__device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, bool f32,
+                                          int part, int nparts) {
   const bool valid = r < g.rows;
   const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   float v[32];
+  const int per = BN / 32 / nparts;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = part * per; c < (part + 1) * per; ++c) {
     tmem_ld32(taddr + 32 * c, v);
     if (!valid) continue;
     if (F8) dequant32(v, sa, g.b_scale + n_idx * BN + 32 * c);
@@ -91,7 +99,8 @@ __device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int
 }
 
 template <bool F8>
-__device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
+__device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, int part,
+                                        int nparts) {
   const bool valid = r < g.rows;
   const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   float v[32];
@@ -99,7 +108,7 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
     const int which = n_idx / 12;            // 0 q, 1 k, 2 v
     const int head0 = (n_idx % 12) * 2;
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int hh = part; hh < 2; hh += nparts) {
       const int head = head0 + hh;
       const uint32_t tcol = taddr + hh * 128;
       const long long bh = (long long)b * kHeads + head;
@@ -154,8 +163,9 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
     const int chunk = n_idx - g.b_split;     // 128 hidden units: gate cols 0..127, up cols 128..255
     __nv_bfloat16* dst = g.a_out + ((long long)b * g.rows + r) * kOutK + kDim + chunk * 128;
     float u[32];
+    const int per = 4 / nparts;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = part * per; c < (part + 1) * per; ++c) {
       tmem_ld32(taddr + 32 * c, v);
       tmem_ld32(taddr + 128 + 32 * c, u);
       if (!valid) continue;
@@ -176,7 +186,8 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
 }
 
 template <int BN, bool F8>
-__device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx) {
+__device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, int part,
+                                          int nparts) {
   const bool valid = r < g.rows;
   const float sa = F8 && valid ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
   const int grow = g.x_row0 + r;
@@ -184,8 +195,9 @@ __device__ __forceinline__ void epi_resid(uint32_t taddr, const GemmArgs& g, int
   const float* gate = g.mod + (long long)mode * 3 * kDim + 2 * kDim + n_idx * BN;
   float* xr = g.x + ((long long)b * g.x_bstride + grow) * kDim + n_idx * BN;
   float v[32];
+  const int per = BN / 32 / nparts;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = part * per; c < (part + 1) * per; ++c) {
     tmem_ld32(taddr + 32 * c, v);
     if (!valid) continue;
     if (F8) dequant32(v, sa, g.b_scale + n_idx * BN + 32 * c);
@@ -321,10 +333,10 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&acc_full[acc], acc_phase, 0x104)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (EPI == kEpiF32) epi_store<BN, false>(taddr, g, b, r, n_idx, true);
-      else if (EPI == kEpiBF16) epi_store<BN, false>(taddr, g, b, r, n_idx, false);
-      else if (EPI == kEpiQKV) epi_qkv<false>(taddr, g, b, r, n_idx);
-      else epi_resid<BN, false>(taddr, g, b, r, n_idx);
+      if (EPI == kEpiF32) epi_store<BN, false>(taddr, g, b, r, n_idx, true, 0, 1);
+      else if (EPI == kEpiBF16) epi_store<BN, false>(taddr, g, b, r, n_idx, false, 0, 1);
+      else if (EPI == kEpiQKV) epi_qkv<false>(taddr, g, b, r, n_idx, 0, 1);
+      else epi_resid<BN, false>(taddr, g, b, r, n_idx, 0, 1);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -375,11 +387,16 @@ struct PairCfg {
   static constexpr int kTileBytes = kStages * kStage;
   static constexpr int kSmem = kTileBytes + 1024 + 256;
   static constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
-  static constexpr int kThreads = 192;
+  // Epilogue warps: two per TMEM lane quarter, each taking half of the
+  // tile's columns, so that one warp's TMEM and global latencies overlap the
+  // other's work (the e4m3 main loop is short enough to wait on a single
+  // warp per quarter).
+  static constexpr int kEpiWarps = KLEIN_PAIR_EPI_WARPS;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
 };
 
 template <int EPI, bool F8>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(PairCfg::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const GemmArgs g) {
   using Cfg = PairCfg;
@@ -403,7 +420,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 256);
+      mbar_init(&acc_empty[a], 2 * 32 * Cfg::kEpiWarps);
     }
     fence_barrier_init();
     tma_prefetch_desc(&map_a);
@@ -486,6 +503,8 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;
+    const int nparts = Cfg::kEpiWarps / 4;
+    const int part = (warp - 2) / 4;
     int it = 0;
     for (int tile = pair; tile < total; tile += npairs, ++it) {
       const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
@@ -497,9 +516,9 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&acc_full[acc], acc_phase, 0x114)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (EPI == kEpiF32) epi_store<256, F8>(taddr, g, b, r, n_idx, true);
-      else if (EPI == kEpiQKV) epi_qkv<F8>(taddr, g, b, r, n_idx);
-      else epi_resid<256, F8>(taddr, g, b, r, n_idx);
+      if (EPI == kEpiF32) epi_store<256, F8>(taddr, g, b, r, n_idx, true, part, nparts);
+      else if (EPI == kEpiQKV) epi_qkv<F8>(taddr, g, b, r, n_idx, part, nparts);
+      else epi_resid<256, F8>(taddr, g, b, r, n_idx, part, nparts);
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
     }
