@@ -46,12 +46,12 @@ WORKLOADS = {
 # measured bf16 peak times the nominal dense ratio (4.5 / 2.25 PFLOP/s).
 FP8_OVER_BF16 = 2.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum of the in-projection GEMM
-# (gemm_pair_kernel<2>), mean over the first 42 launches of a t2i denoise, from
-# one ncu capture of the current kernel (its summary is kept with the other
-# kernel profiles). Must be re-captured (or set to None) whenever that kernel
-# changes.
-GEMM_IN_TRAFFIC_BYTES = 314.35e6
+# dram__bytes_read.sum + dram__bytes_write.sum of the bf16 in-projection GEMM
+# (gemm_pair_kernel<2, 0>, eight epilogue warps), mean over the first 42
+# launches of a t2i denoise, from one ncu capture of the current kernel (its
+# summary is kept with the other kernel profiles). Must be re-captured (or set
+# to None) whenever that kernel changes.
+GEMM_IN_TRAFFIC_BYTES = 314.95e6
 
 
 def load_peaks():
