@@ -137,7 +137,9 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
       }
       const float rs = rsqrtf(ss * (1.0f / kHeadDim) + kRmsEps);
-      const float2* rope = g.rope + (long long)(valid ? r : 0) * kPairs;
+      // (cos, sin) of two pairs and four norm weights per 16-byte load
+      const float4* rope4 = reinterpret_cast<const float4*>(g.rope + (long long)(valid ? r : 0) * kPairs);
+      const float4* w4 = reinterpret_cast<const float4*>(w);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tcol + 32 * c, v);
@@ -145,12 +147,14 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
         if (F8) dequant32(v, sa, sb + 32 * c);
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 32; i += 4) {
           const int d = 32 * c + i;
-          const float y0 = v[i] * rs * __ldg(w + d);
-          const float y1 = v[i + 1] * rs * __ldg(w + d + 1);
-          const float2 cs = rope[d >> 1];
+          const float4 wn = __ldg(w4 + (d >> 2));
+          const float4 cs = __ldg(rope4 + (d >> 2));  // pairs d/2 and d/2 + 1
+          const float y0 = v[i] * rs * wn.x, y1 = v[i + 1] * rs * wn.y;
+          const float y2 = v[i + 2] * rs * wn.z, y3 = v[i + 3] * rs * wn.w;
           pk[i >> 1] = pack_bf16(y0 * cs.x - y1 * cs.y, y0 * cs.y + y1 * cs.x);
+          pk[(i >> 1) + 1] = pack_bf16(y2 * cs.z - y3 * cs.w, y2 * cs.w + y3 * cs.z);
         }
         __nv_bfloat16* o = dst + 32 * c;
         store16(o, pk[0], pk[1], pk[2], pk[3]);
