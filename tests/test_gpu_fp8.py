@@ -204,3 +204,35 @@ def test_fp8_denoise_matches_oracle(kb):
     ref = o.denoise(fp8.QuantizedModel(m), lat, text, rl, o.positions(40, (6, 6), refs), 3)
     assert cosine(host(x), ref) >= 0.999
     assert max_err_ratio(host(x), ref) <= 5e-2
+
+
+@pytest.mark.parametrize("batch,n_txt,grid,refs", [(1, 512, (64, 64), ()), (1, 512, (64, 64), ((64, 64),))])
+def test_fp8_block_full_size_sampled_rows(kb, fp8_weights, batch, n_txt, grid, refs):
+    # the 1024x1024 text-to-image (4608 rows) and edit (8704 rows) joint
+    # blocks in FP8; the oracle evaluates a sample of output rows, every row
+    # supplying keys and values
+    wq, _, wd = fp8_weights
+    n_img = grid[0] * grid[1]
+    n_ref = sum(h * ww for h, ww in refs)
+    n_total = n_txt + n_img + n_ref
+    seq = kb.make_seq(batch, n_txt, grid[0], grid[1], refs)
+    x = ki.tokens(1, f"fp8block.large.{n_total}", batch, n_total)
+    mod = ki.modulation_vectors(1, f"fp8block.large.{n_total}")
+    xd = to_f32(x)
+    pos = torch.empty((n_total, 4), dtype=torch.float32, device="cuda")
+    kb.klein_positions(seq, pos)
+    ws = workspace(kb.klein_block_workspace_size(batch, n_total))
+    kb.klein_block_forward(wd, xd, n_txt, n_img, pos, to_f32(mod), ws)
+    torch.cuda.synchronize()
+    got = host(xd)
+    rows = np.unique(np.concatenate([np.arange(0, n_total, 331), [0, n_txt - 1, n_txt, n_txt + n_img - 1,
+                                                                 n_total - 1]]))
+    rows = rows[rows < n_total]
+    ref = o.block(x, o.positions(n_txt, grid, refs), o.mode_of_rows(n_txt, n_img, n_ref),
+                  mod.astype(np.float64), wq, rows=rows)
+    g = got[:, rows]
+    d_got, d_ref = g - x[:, rows], ref - x[:, rows]
+    assert np.all(np.isfinite(g))
+    assert rms(d_got - d_ref) / rms(d_ref) <= 3e-2
+    assert cosine(d_got, d_ref) >= 0.999
+    assert max_err_ratio(g, ref) <= FP8_MAX_ERR, max_err_ratio(g, ref)
