@@ -267,11 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mvt, const AttnArgs& a,
                      cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
+  static bool configured[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  if (!configured[dev]) {
     if (cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
       return -1;
-    configured = true;
+    configured[dev] = true;
   }
   if (a.rows <= 0 || a.batch <= 0) return 0;
   dim3 grid((a.rows + 255) / 256, a.heads, a.batch);

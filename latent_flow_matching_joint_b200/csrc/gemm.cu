@@ -358,12 +358,14 @@ __global__ void __launch_bounds__(192, 1)
 template <int BN, int EPI>
 static int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
   using Cfg = GemmCfg<BN>;
-  static bool configured = false;
-  if (!configured) {
+  static bool configured[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  if (!configured[dev]) {
     if (cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
         cudaSuccess)
       return -1;
-    configured = true;
+    configured[dev] = true;
   }
   const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
   if (total <= 0) return 0;
@@ -541,7 +543,10 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
 template <int EPI, bool F8>
 static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, cudaStream_t s) {
   using Cfg = PairCfg;
-  static int max_pairs = 0;
+  static int max_pairs_dev[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  int& max_pairs = max_pairs_dev[dev];
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -133,6 +133,11 @@ int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_
 
 int launch_wait_probe(unsigned long long limit_ns, cudaStream_t stream);
 int num_sms();
+// Index of the current device, or -1 if it is outside [0, kMaxDevices).
+// Per-function launch settings (shared-memory opt-in, cluster occupancy) are
+// per device, so the launchers keep them per device index.
+constexpr int kMaxDevices = 64;
+int current_device();
 
 // Host-side count of kernels launched by this library (all entry points).
 void note_launch();

@@ -470,12 +470,14 @@ int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_
                 long long y_stride, int act_silu, const float* add, cudaStream_t s) {
   if (n_vec < 1 || n_vec > kMaxVec || (k % 8) != 0) return -2;
   const size_t smem = sizeof(float) * n_vec * k;
-  static bool configured = false;
-  if (!configured) {
+  static bool configured[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  if (!configured[dev]) {
     if (cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxVec * kDim * 4) !=
         cudaSuccess)
       return -1;
-    configured = true;
+    configured[dev] = true;
   }
   gemv_kernel<<<(n_out + 7) / 8, 256, smem, s>>>(w, n_out, k, x, n_vec, x_stride, y, y_stride, act_silu, add);
   note_launch();

@@ -34,6 +34,12 @@ static int cuda_fail(const char* what) {
 static long long g_launches = 0;
 void note_launch() { ++g_launches; }
 
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 int num_sms() {
   static int cached[64] = {0};
   int dev = 0;
