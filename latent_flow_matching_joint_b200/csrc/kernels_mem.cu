@@ -85,8 +85,11 @@ __device__ __forceinline__ void e4m3_row_scales(float amax, float& inv, float& s
   scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
 }
 
-// modLN with the output quantised: one warp per row, as modln_kernel.
-__global__ void __launch_bounds__(256, 2) modln_e4m3_kernel(const float* __restrict__ x, long long x_bstride,
+// modLN with the output quantised: one warp per row, as modln_kernel. The
+// modulated row stays in registers between the row maximum and the codes
+// (one block of 8 warps per SM: 8 x 32 lanes x 24 x 16 bytes of loads in
+// flight per SM still cover the HBM latency).
+__global__ void __launch_bounds__(256, 1) modln_e4m3_kernel(const float* __restrict__ x, long long x_bstride,
                                                          int x_row0, uint32_t* __restrict__ codes,
                                                          float* __restrict__ scale, int batch, int rows,
                                                          int n_txt, int n_img, const float* __restrict__ mod,
@@ -121,20 +124,19 @@ __global__ void __launch_bounds__(256, 2) modln_e4m3_kernel(const float* __restr
   const int m = mode_of_row(grow, n_txt, n_img);
   const float4* shift = reinterpret_cast<const float4*>(mod + m * mod_stride);
   const float4* scl = reinterpret_cast<const float4*>(mod + m * mod_stride + kDim);
-  // The modulated rows are formed twice, identically: once for the row
-  // maximum and once for the codes, so that only x stays in registers.
   float amax = 0.f;
 #pragma unroll
   for (int t = 0; t < kVec; ++t) {
     const int c4 = lane + 32 * t;
     const float4 sc = __ldg(scl + c4);
     const float4 sh = __ldg(shift + c4);
-    const float4 e = v[t];
-    const float h0 = fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x);
-    const float h1 = fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y);
-    const float h2 = fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z);
-    const float h3 = fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w);
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+    float4 e = v[t];
+    e.x = fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x);
+    e.y = fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y);
+    e.z = fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z);
+    e.w = fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(e.x), fabsf(e.y)), fmaxf(fabsf(e.z), fabsf(e.w))));
+    v[t] = e;
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -142,15 +144,8 @@ __global__ void __launch_bounds__(256, 2) modln_e4m3_kernel(const float* __restr
   e4m3_row_scales(amax, inv, s);
 #pragma unroll
   for (int t = 0; t < kVec; ++t) {
-    const int c4 = lane + 32 * t;
-    const float4 sc = __ldg(scl + c4);
-    const float4 sh = __ldg(shift + c4);
     const float4 e = v[t];
-    const float h0 = fmaf((e.x - mean) * rstd, 1.f + sc.x, sh.x);
-    const float h1 = fmaf((e.y - mean) * rstd, 1.f + sc.y, sh.y);
-    const float h2 = fmaf((e.z - mean) * rstd, 1.f + sc.z, sh.z);
-    const float h3 = fmaf((e.w - mean) * rstd, 1.f + sc.w, sh.w);
-    dst[c4] = pack_e4m3x4(__fmul_rn(h0, inv), __fmul_rn(h1, inv), __fmul_rn(h2, inv), __fmul_rn(h3, inv));
+    dst[lane + 32 * t] = pack_e4m3x4(__fmul_rn(e.x, inv), __fmul_rn(e.y, inv), __fmul_rn(e.z, inv), __fmul_rn(e.w, inv));
   }
   if (lane == 0) scale[(long long)b * rows + i] = s;
 }
