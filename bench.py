@@ -52,7 +52,7 @@ FP8_OVER_BF16 = 2.0
 # launches of a t2i denoise, from one ncu capture of the current kernel (its
 # summary is kept with the other kernel profiles). Must be re-captured (or set
 # to None) whenever that kernel changes.
-GEMM_IN_TRAFFIC_BYTES = 314.38e6
+GEMM_IN_TRAFFIC_BYTES = None
 
 
 def load_peaks():

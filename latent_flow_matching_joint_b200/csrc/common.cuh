@@ -77,7 +77,10 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast reciprocal-based division (a few ulp,
+// far below the bf16 rounding of every result it feeds); for g below about
+// -87 the denominator passes 2^126 and the quotient is 0, the function's limit.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Two-wide fp32 arithmetic (one instruction for a pair of lanes' values):
 // (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1), and (d0, d1) += (a0, a1).
