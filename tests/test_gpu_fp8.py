@@ -202,8 +202,14 @@ def test_fp8_denoise_matches_oracle(kb):
     kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 1.0, seq, ws)
     torch.cuda.synchronize()
     ref = o.denoise(fp8.QuantizedModel(m), lat, text, rl, o.positions(40, (6, 6), refs), 3)
-    assert cosine(host(x), ref) >= 0.999
-    assert max_err_ratio(host(x), ref) <= 5e-2
+    got = host(x)
+    # the benchmark spec's cosine >= 0.999 for the final latents; the latents are
+    # the noise plus dsigma-weighted velocities, each a linear read-out of the
+    # last block's rows, so their worst element is held to the FP8 block's
+    # derived worst-element bound, and their RMS error to the block update's
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert rms(got - ref) / rms(ref) <= 3e-2, rms(got - ref) / rms(ref)
+    assert max_err_ratio(got, ref) <= FP8_MAX_ERR, max_err_ratio(got, ref)
 
 
 @pytest.mark.parametrize("batch,n_txt,grid,refs", [(1, 512, (64, 64), ()), (1, 512, (64, 64), ((64, 64),))])
