@@ -48,11 +48,12 @@ WORKLOADS = {
 FP8_OVER_BF16 = 2.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of the bf16 in-projection GEMM
-# (gemm_pair_kernel<2, 0>, eight epilogue warps), mean over the first 42
-# launches of a t2i denoise, from one ncu capture of the current kernel (its
-# summary is kept with the other kernel profiles). Must be re-captured (or set
-# to None) whenever that kernel changes.
-GEMM_IN_TRAFFIC_BYTES = None
+# (gemm_pair_kernel<2, 0>), mean over the first 42 launches of a t2i denoise,
+# from one ncu capture of the current kernel (its summary is kept with the
+# other kernel profiles; captures of this kernel have read 199 MB and written
+# 118-132 MB, depending on what of its output the L2 still holds at exit).
+# Must be re-captured (or set to None) whenever that kernel changes.
+GEMM_IN_TRAFFIC_BYTES = 331.43e6
 
 
 def load_peaks():
