@@ -110,3 +110,27 @@ def test_model_create_validation(kb):
     h = ctypes.c_void_p()
     rc = kb.lib.klein_model_create(ctypes.byref(h), ctypes.byref(d))
     assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
+
+
+def test_fp8_argument_errors_before_any_launch(kb):
+    q = kb.lib.klein_quantize_rowwise_e4m3
+    rc = q(None, 4, 16, 256, 512, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
+    rc = q(256, 4, 12, 4096, 8192, None)                 # cols not a multiple of 8
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    rc = q(256, 4, 12296, 1 << 20, 1 << 21, None)        # cols beyond 12288
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    rc = q(264, 4, 16, 4096, 8192, None)                 # src not 16-byte aligned
+    assert kb.STATUS[rc] == "KLEIN_ERR_ALIGN"
+    rc = q(4096, 4, 16, 4096 + 64, 8192, None)           # codes overlap src
+    assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
+    g = kb.lib.klein_op_gemm_e4m3
+    rc = g(256, 512, 1024, 2048, 4096, 10, 200, 128, None)  # N not a multiple of 256
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    rc = g(256, 512, 1024, 2048, 4096, 10, 256, 96, None)   # K not a multiple of 128
+    assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+    # FP8 block weights need both scales
+    bw = kb.KleinBlockWeights(16, 32, 48, 64, 80, None)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1 << 30, None)
+    assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
+    assert b"w_in_scale and w_out_scale" in kb.lib.klein_last_error()
