@@ -70,6 +70,19 @@ __device__ __forceinline__ void dequant32(float* v, float sa, const float* sb) {
 
 // part / nparts: this warp's share of the tile's columns when several
 // epilogue warps serve the same TMEM lane quarter.
+// The output channel's weight scale alone (the row's scale folded elsewhere).
+__device__ __forceinline__ void colscale32(float* v, const float* sb) {
+  const float4* s4 = reinterpret_cast<const float4*>(sb);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = __ldg(s4 + i);
+    v[4 * i + 0] *= t.x;
+    v[4 * i + 1] *= t.y;
+    v[4 * i + 2] *= t.z;
+    v[4 * i + 3] *= t.w;
+  }
+}
+
 template <int BN, bool F8>
 __device__ __forceinline__ void epi_store(uint32_t taddr, const GemmArgs& g, int b, int r, int n_idx, bool f32,
                                           int part, int nparts) {
@@ -132,15 +145,18 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
       }
       const float* w = which == 0 ? g.q_norm : g.k_norm;
       __nv_bfloat16* dst = (which == 0 ? g.q : g.k) + (bh * g.rows_pad + r) * kHeadDim;
+      // e4m3: the head's values are sa * acc * sb; the row scale sa is folded
+      // into the RMS normalisation (sa * rsqrt(sa^2 * mean((acc sb)^2) + eps))
       float ss = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tcol + 32 * c, v);
-        if (F8) dequant32(v, sa, sb + 32 * c);
+        if (F8) colscale32(v, sb + 32 * c);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
       }
-      const float rs = rsqrtf(ss * (1.0f / kHeadDim) + kRmsEps);
+      const float rs = F8 ? sa * rsqrtf(sa * sa * ss * (1.0f / kHeadDim) + kRmsEps)
+                          : rsqrtf(ss * (1.0f / kHeadDim) + kRmsEps);
       // (cos, sin) of two pairs and four norm weights per 16-byte load
       const float4* rope4 = reinterpret_cast<const float4*>(g.rope + (long long)(valid ? r : 0) * kPairs);
       const float4* w4 = reinterpret_cast<const float4*>(w);
@@ -148,7 +164,7 @@ __device__ __forceinline__ void epi_qkv(uint32_t taddr, const GemmArgs& g, int b
       for (int c = 0; c < 4; ++c) {
         tmem_ld32(tcol + 32 * c, v);
         if (!valid) continue;
-        if (F8) dequant32(v, sa, sb + 32 * c);
+        if (F8) colscale32(v, sb + 32 * c);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
