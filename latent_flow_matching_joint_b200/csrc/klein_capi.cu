@@ -539,7 +539,7 @@ int klein_model_create(klein_model** out, const klein_model_desc* d) {
 void klein_model_destroy(klein_model* m) { delete m; }
 
 size_t klein_stack_workspace_size(const klein_seq* seq) {
-  int ni, nr, nt;
+  int ni = 0, nr = 0, nt = 0;
   if (check_seq(seq, &ni, &nr, &nt)) return 0;
   return carve_stack(nullptr, seq->batch, nt, ni, nr).bytes;
 }
@@ -746,7 +746,7 @@ static int check_stack_args(const klein_model* m, const void* latents, const voi
 int klein_stack_forward(const klein_model* m, const float* latents, const void* text, const float* refs,
                         float sigma, float sigma_next, const klein_seq* seq, float* v_out, void* ws,
                         size_t ws_bytes, void* stream) {
-  int ni, nr, nt;
+  int ni = 0, nr = 0, nt = 0;
   int rc = check_stack_args(m, latents, text, refs, seq, ws, ws_bytes, &ni, &nr, &nt);
   if (rc) return rc;
   if (!v_out || !aligned16(v_out)) return fail(KLEIN_ERR_ALIGN, "v_out must be a 16-byte aligned device pointer");
@@ -757,7 +757,7 @@ int klein_stack_forward(const klein_model* m, const float* latents, const void* 
 
 int klein_denoise(const klein_model* m, float* latents, const void* text, const float* refs, int steps, float cfg,
                   float shift, const klein_seq* seq, float* x0_out, void* ws, size_t ws_bytes, void* stream) {
-  int ni, nr, nt;
+  int ni = 0, nr = 0, nt = 0;
   int rc = check_stack_args(m, latents, text, refs, seq, ws, ws_bytes, &ni, &nr, &nt);
   if (rc) return rc;
   if (steps < 1 || steps > 1000) return fail(KLEIN_ERR_INVALID_ARG, "steps out of range");
