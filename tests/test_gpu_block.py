@@ -10,7 +10,7 @@ torch = pytest.importorskip("torch")
 
 import klein_inputs as ki  # noqa: E402
 import oracle as o  # noqa: E402
-from gpu_util import cosine, host, max_err_ratio, to_bf16, to_f32, upload_block, workspace  # noqa: E402
+from gpu_util import cosine, host, max_err_ratio, to_f32, upload_block, workspace  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 

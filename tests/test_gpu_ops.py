@@ -22,7 +22,7 @@ def kb():
     return kb
 
 
-from gpu_util import cosine, host, max_err_ratio, rms, to_bf16, to_f32, workspace  # noqa: E402
+from gpu_util import cosine, host, rms, to_bf16, to_f32  # noqa: E402
 
 
 # ------------------------------------------------------------------ GEMM
