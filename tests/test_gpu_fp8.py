@@ -203,7 +203,7 @@ def test_fp8_denoise_matches_oracle(kb):
     torch.cuda.synchronize()
     ref = o.denoise(fp8.QuantizedModel(m), lat, text, rl, o.positions(40, (6, 6), refs), 3)
     got = host(x)
-    # the benchmark spec's cosine >= 0.999 for the final latents; the latents are
+    # the final latents keep cosine >= 0.999 to the oracle's; they are
     # the noise plus dsigma-weighted velocities, each a linear read-out of the
     # last block's rows, so their worst element is held to the FP8 block's
     # derived worst-element bound, and their RMS error to the block update's
