@@ -10,7 +10,7 @@ same size (1.3916 TFLOP) is timed alone in the same run, before the denoise,
 and reported as `joint_block`.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload t2i|edit|cfg2048|block] [--precision bf16|fp8]
+                    [--workload t2i|edit|cfg2048|block|memory] [--precision bf16|fp8]
                     [--no-cpu-baseline]
 """
 from __future__ import annotations
@@ -342,12 +342,98 @@ def run_block_only(args):
     return 0
 
 
+def run_memory(args):
+    """The memory-bound kernels against the measured HBM bandwidth: modLN
+    (bf16 and e4m3 outputs), the standalone RoPE and the Euler update over a
+    size sweep. Each size rotates over enough input sets that every call reads
+    from HBM (sets x bytes > L2) where the size allows; the smallest Euler
+    sizes are launch-bound and L2-resident by nature."""
+    import torch
+    import latent_flow_matching_joint_b200 as kb
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    l2 = 126e6
+    g = torch.Generator(device=dev).manual_seed(0)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, nsets, iters=40):
+        for i in range(max(args.warmup, 3)):
+            fn(i % nsets)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(iters):
+            fn(i % nsets)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters * 1e3  # us
+
+    def sets_for(nbytes):
+        return max(2, min(8, int(3 * l2 // max(nbytes, 1)) + 1))
+
+    results = []
+
+    def add(kernel, size, nbytes, us):
+        gbs = nbytes / us / 1e3
+        results.append({"kernel": kernel, "size": size, "bytes": nbytes, "us": us, "GB/s": gbs,
+                        "frac_of_hbm": gbs / peaks["hbm"]})
+
+    mod = 0.5 * torch.randn(3, 3, DIM, generator=g, device=dev)
+    for batch, rows in ((1, 4608), (1, 8704), (2, 16944)):
+        nbytes_in = batch * rows * DIM * 4
+        ns = sets_for(nbytes_in)
+        xs = [torch.randn(batch, rows, DIM, generator=g, device=dev) for _ in range(ns)]
+        h = torch.empty(batch, rows, DIM, device=dev, dtype=torch.bfloat16)
+        codes = torch.empty(batch, rows, DIM, device=dev, dtype=torch.uint8)
+        sc = torch.empty(batch, rows, device=dev)
+        us = timed(lambda i: kb.klein_op_modln(xs[i], 0, rows, 512, rows - 512, mod, h), ns)
+        add("modln (fp32 x -> bf16 h)", f"{batch}x{rows} rows", batch * rows * DIM * 6, us)
+        us = timed(lambda i: kb.klein_op_modln_e4m3(xs[i], 0, rows, 512, rows - 512, mod, codes, sc), ns)
+        add("modln_e4m3 (fp32 x -> e4m3 h + row scale)", f"{batch}x{rows} rows", batch * rows * (DIM * 5 + 4), us)
+        del xs, h, codes, sc
+    for rows in (4608, 16944):
+        pos = torch.arange(rows * 4, device=dev, dtype=torch.float32).view(rows, 4) % 97  # any positions
+        table = torch.empty(rows, 64, 2, device=dev)
+        kb.klein_op_rope_table(pos, table)
+        nbytes = rows * DIM * 2 * 2
+        ns = sets_for(nbytes)
+        ins = [torch.randn(rows, 24, 128, generator=g, device=dev).to(torch.bfloat16) for _ in range(ns)]
+        out = torch.empty(rows, 24, 128, device=dev, dtype=torch.bfloat16)
+        us = timed(lambda i: kb.klein_op_rope(ins[i], out, table), ns)
+        add("rope (bf16 [rows][24][128] in -> out)", f"{rows} rows", nbytes, us)
+        del ins, out
+    for n in (4096 * 128, 16384 * 128 * 2, 1 << 24, 1 << 26):
+        ns = sets_for(n * 8)
+        xs = [torch.randn(n, generator=g, device=dev) for _ in range(ns)]
+        vc = [torch.randn(n, generator=g, device=dev) for _ in range(ns)]
+        vu = torch.randn(n, generator=g, device=dev)
+        us = timed(lambda i: kb.klein_op_euler(xs[i], vc[i], None, -0.01), ns)
+        add("euler (x += dsigma v)", f"{n} elements", n * 12, us)
+        us = timed(lambda i: kb.klein_op_euler(xs[i], vc[i], vu, -0.01, 3.5), ns)
+        add("euler with CFG", f"{n} elements", n * 16, us)
+        del xs, vc, vu
+    rc, _, msg = kb.klein_device_status()
+    if rc != 0:
+        raise RuntimeError(msg)
+    first = results[0]
+    print(json.dumps({"metric": "memory-bound kernels: achieved GB/s against the measured HBM copy bandwidth",
+                      "value": first["GB/s"], "unit": "GB/s", "peak": peaks["hbm"],
+                      "peak_source": f"{peaks['source']} hbm_gbs", "dtype": "f32/bf16/e4m3",
+                      "config": {"workload": "modLN, RoPE, Euler size sweep; inputs rotated over > L2 where the "
+                                             "size allows"},
+                      "results": results}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
     if args.workload == "block":
         return run_block_only(args)
+    if args.workload == "memory":
+        return run_memory(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -538,7 +624,7 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=tuple(WORKLOADS) + ("block",), default="t2i")
+    ap.add_argument("--workload", choices=tuple(WORKLOADS) + ("block", "memory"), default="t2i")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--precision", choices=tuple(DTYPES), default="bf16",
                     help="block GEMM operands: bf16, or rowwise FP8 (e4m3 codes, one scale per row)")

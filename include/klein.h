@@ -25,7 +25,8 @@
  *     message (thread-local, valid until the next call on that thread).
  *   - A failed kernel launch returns KLEIN_ERR_CUDA. A device-side wait that
  *     gave up (no progress for the wait limit) is recorded on the device and
- *     reported by klein_device_status() as KLEIN_ERR_TIMEOUT.
+ *     reported by klein_sync(stream) or klein_device_status() as
+ *     KLEIN_ERR_TIMEOUT.
  *   - Device pointers must be 16-byte aligned. The model width is fixed at
  *     KLEIN_DIM = 3072, 24 heads of 128.
  *   - bf16 = IEEE bfloat16 stored as uint16; all matrices are row-major.
@@ -77,6 +78,13 @@ long long klein_launch_count(void);
  * bounded wait gave up, KLEIN_ERR_CUDA on a CUDA error. `site` (may be NULL)
  * receives the code of the wait that gave up. */
 int klein_device_status(unsigned* site);
+
+/* Waits for the work queued on `stream`, then reports as klein_device_status
+ * does (without synchronising other streams): KLEIN_OK, KLEIN_ERR_TIMEOUT when
+ * a bounded wait gave up, KLEIN_ERR_CUDA on a CUDA error. The device error
+ * word is per device: a wait that gave up in this library's work on another
+ * stream of the same device is reported (and cleared) here too. */
+int klein_sync(void* stream);
 
 /* Sets the bound (nanoseconds) of every device-side wait; default 2 s. */
 int klein_set_wait_limit_ns(unsigned long long ns);

@@ -64,6 +64,7 @@ _SIGS = {
     "klein_version": (c_int, []),
     "klein_launch_count": (c_longlong, []),
     "klein_device_status": (c_int, [POINTER(c_uint)]),
+    "klein_sync": (c_int, [c_void_p]),
     "klein_set_wait_limit_ns": (c_int, [c_ulonglong]),
     "klein_wait_probe": (c_int, [c_ulonglong, c_void_p]),
     "klein_profile_begin": (c_int, [c_int]),
@@ -165,6 +166,13 @@ def klein_device_status():
     site = c_uint()
     rc = lib.klein_device_status(ctypes.byref(site))
     return rc, site.value, lib.klein_last_error().decode(errors="replace")
+
+
+def klein_sync(stream=None):
+    """(status, message) after the stream's queued work: 0, or KLEIN_ERR_TIMEOUT
+    when a bounded device wait gave up (read and cleared)."""
+    rc = lib.klein_sync(_stream(stream))
+    return rc, lib.klein_last_error().decode(errors="replace")
 
 
 def klein_set_wait_limit_ns(ns: int):

@@ -352,8 +352,8 @@ int klein_version(void) { return 102; }
 
 long long klein_launch_count(void) { return g_launches; }
 
-int klein_device_status(unsigned* site) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail("cudaDeviceSynchronize");
+// Reads and clears the device error word that bounded waits write.
+static int take_device_error(unsigned* site) {
   unsigned err = 0, where = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&err, g_klein_error, sizeof(err)) != cudaSuccess ||
       cudaMemcpyFromSymbol(&where, g_klein_error_site, sizeof(where)) != cudaSuccess ||
@@ -365,6 +365,17 @@ int klein_device_status(unsigned* site) {
   if (err) return fail(KLEIN_ERR_CUDA, "device error bits 0x%x at site 0x%x", err, where);
   g_msg[0] = 0;
   return KLEIN_OK;
+}
+
+int klein_device_status(unsigned* site) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail("cudaDeviceSynchronize");
+  return take_device_error(site);
+}
+
+int klein_sync(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return cuda_fail("cudaStreamSynchronize");
+  return take_device_error(nullptr);
 }
 
 int klein_set_wait_limit_ns(unsigned long long ns) {

@@ -191,3 +191,14 @@ def test_wait_probe_reports_timeout(kb):
     a = torch.ones(4, device="cuda")
     assert float(a.sum()) == 4.0
     assert kb.klein_device_status()[0] == 0
+
+
+def test_sync_reports_timeout_on_its_stream(kb):
+    s = torch.cuda.Stream()
+    assert kb.klein_sync(s.cuda_stream)[0] == 0
+    with torch.cuda.stream(s):
+        kb.klein_wait_probe(2_000_000, s.cuda_stream)  # 2 ms, nothing ever arrives
+    rc, msg = kb.klein_sync(s.cuda_stream)
+    assert kb.STATUS[rc] == "KLEIN_ERR_TIMEOUT", msg
+    assert kb.klein_sync(s.cuda_stream)[0] == 0     # read and cleared
+    assert kb.klein_device_status()[0] == 0
