@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <new>
 
 #include "../../include/klein.h"
@@ -31,8 +32,9 @@ static int cuda_fail(const char* what) {
   return fail(KLEIN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-static long long g_launches = 0;
-void note_launch() { ++g_launches; }
+// Launch counter over all entry points (host threads may launch concurrently).
+static std::atomic<long long> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int current_device() {
   int dev = 0;
@@ -41,10 +43,9 @@ int current_device() {
 }
 
 int num_sms() {
-  static int cached[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
+  static int cached[kMaxDevices] = {0};
+  int dev = current_device();
+  if (dev < 0) dev = 0;
   if (!cached[dev]) {
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
