@@ -258,7 +258,11 @@ typedef struct klein_model klein_model;
 int klein_model_create(klein_model** out, const klein_model_desc* desc);
 void klein_model_destroy(klein_model* m);
 
-/* Workspace bytes for klein_stack_forward / klein_denoise on `seq`. */
+/* Workspace bytes for klein_stack_forward / klein_denoise on `seq`. A
+ * workspace serves one call at a time: calls that overlap on the device
+ * (different streams) need their own. klein_denoise keeps state in it across
+ * its steps (the projected text; for the base model, the text and reference
+ * streams' stage-1 output, computed at the first step and reused after it). */
 size_t klein_stack_workspace_size(const klein_seq* seq);
 
 /* One denoiser call ([blog]; [guide] "Inside the transformer", "What step
