@@ -1,0 +1,116 @@
+"""Pins for the oracle's NVFP4 quantisation (e2m1 values, e4m3 block scales,
+fp32 tensor scale).
+
+The e2m1 encoder is checked against brute force (the nearest of the eight
+magnitudes, ties to the even code) on every midpoint and a dense grid, and
+against worked values; the block quantiser against what its definition fixes:
+each block's largest value lands on 6 while its scale is a normal e4m3 value,
+the error of a 1-bit mantissa, the coarser subnormal-scale regime of blocks far
+below the tensor maximum, exact round trips of representable tensors, the zero
+tensor, and scales that follow each 16-value block rather than the row.
+"""
+import numpy as np
+import pytest
+
+from oracle import fp8, nvfp4
+
+MAGS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _brute(x):
+    a = np.minimum(np.abs(x), 6.0)
+    d = np.abs(a[:, None] - MAGS[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = np.where(np.isclose(d, best, rtol=0, atol=0), np.arange(8)[None, :], 99)
+    even = np.where(cand % 2 == 0, cand, 99).min(axis=1)
+    code = np.where(even < 99, even, cand.min(axis=1))
+    return (code | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def test_decode_table():
+    c = np.arange(16, dtype=np.uint8)
+    want = np.concatenate([MAGS, -MAGS])
+    np.testing.assert_array_equal(nvfp4.e2m1_decode(c), want)
+
+
+def test_encode_matches_brute_force():
+    mids = (MAGS[:-1] + MAGS[1:]) / 2
+    grid = np.linspace(-8, 8, 4097)
+    x = np.concatenate([mids, -mids, MAGS, -MAGS, grid, [7.0, 100.0, -1e9]]).astype(np.float32)
+    np.testing.assert_array_equal(nvfp4.e2m1_encode(x), _brute(x.astype(np.float64)))
+
+
+def test_encode_worked_values():
+    x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -3.0, -0.0, np.inf], np.float32)
+    want = [0, 2, 2, 4, 4, 6, 6, 7, 8 | 5, 8, 7]
+    assert nvfp4.e2m1_encode(x).tolist() == want
+
+
+def test_block_max_lands_on_six_and_error_bound():
+    # block magnitudes spread over 2^8, so every block scale is a normal e4m3 value
+    rng = np.random.default_rng(5)
+    mag = np.exp(rng.uniform(-2.7, 2.7, (32, 8, 1)))      # 8 blocks per row, each its own scale
+    x = (rng.standard_normal((32, 8, 16)) * mag).astype(np.float32).reshape(32, 128)
+    codes, sb, g = nvfp4.quantize(x)
+    assert codes.shape == (32, 128) and sb.shape == (32, 8) and g.dtype == np.float32
+    dec = nvfp4.e2m1_decode(codes).reshape(32, 8, 16)
+    assert np.all(np.max(np.abs(dec), axis=-1) == 6.0)
+    step = fp8.e4m3_decode(sb) * np.float64(g)
+    amax = np.max(np.abs(x.reshape(32, 8, 16)), axis=-1)
+    # the block scale follows the block's own maximum (within the e4m3 rounding of the scale)
+    np.testing.assert_allclose(step * 6.0, amax, rtol=2.0 ** -4 + 1e-6)
+    assert np.all((sb >> 3) & 0xF > 0)                       # normal e4m3 scales only
+    err = np.abs(nvfp4.dequantize(codes, sb, g) - x).reshape(32, 8, 16)
+    bound = np.maximum(0.25 * np.abs(x.reshape(32, 8, 16)), 0.25 * step[..., None]) * (1 + 1e-6)
+    assert np.all(err <= bound)
+
+
+def test_blocks_far_below_the_tensor_maximum():
+    # the tensor scale puts the largest block's scale at 448; a block 2^17
+    # below it needs a scale of about 448 * 2^-17 < 2^-6, e4m3's smallest
+    # normal: the scale is then a subnormal e4m3 value (steps of 2^-9), coarse
+    # enough that the block's maximum may miss 6, and values that the scale's
+    # rounding pushes past 6 saturate
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((1, 64)).astype(np.float32)
+    x[0, :16] *= np.float32(2.0 ** 17)
+    codes, sb, g = nvfp4.quantize(x)
+    assert ((sb[0, 1:] >> 3) & 0xF == 0).all() and ((sb[0, 0] >> 3) & 0xF) > 0
+    dq = nvfp4.dequantize(codes, sb, g)
+    rel = np.abs(dq[0, 16:] - x[0, 16:]) / np.max(np.abs(x[0, 16:]))
+    assert rel.max() <= 0.5
+    np.testing.assert_allclose(dq[0, :16], x[0, :16], rtol=0.25, atol=0.25 * 6 * float(
+        fp8.e4m3_decode(sb[0, 0])) * float(g))
+
+
+def test_exact_round_trip_and_zero_tensor():
+    rng = np.random.default_rng(6)
+    codes = rng.integers(0, 16, (4, 64)).astype(np.uint8)
+    codes[:, ::16] = 7                                       # every block reaches 6
+    sb_vals = fp8.e4m3_decode(rng.integers(0x30, 0x50, (4, 4)).astype(np.uint8))
+    g = np.float32(2.0 ** -5)
+    # tensor scale chosen so that the largest block scale is exactly representable and
+    # 448 * 6 * g equals the tensor's maximum
+    x = (nvfp4.e2m1_decode(codes).reshape(4, 4, 16) * sb_vals[..., None] * np.float64(g)).reshape(4, 64)
+    gq = np.float32(np.max(np.abs(x)) / (448.0 * 6.0))
+    q, sb, g2 = nvfp4.quantize(x.astype(np.float32), g=g)
+    np.testing.assert_array_equal(nvfp4.dequantize(q, sb, g2), x)
+    assert gq > 0
+    z, zs, zg = nvfp4.quantize(np.zeros((2, 32), np.float32))
+    assert zg == 0 and not z.any() and not zs.any()
+
+
+def test_quantised_product_error_is_the_formats():
+    rng = np.random.default_rng(7)
+    a = rng.standard_normal((64, 256)).astype(np.float32)
+    b = rng.standard_normal((48, 256)).astype(np.float32)
+    exact = a.astype(np.float64) @ b.astype(np.float64).T
+    q = nvfp4.fake_quant(a) @ nvfp4.fake_quant(b).T
+    rel = np.sqrt(np.mean((q - exact) ** 2) / np.mean(exact ** 2))
+    # one mantissa bit: about 0.1 relative RMS error per operand, ~0.14 for the product
+    assert 0.05 < rel < 0.2, rel
+
+
+def test_rejects_ragged_rows():
+    with pytest.raises(ValueError):
+        nvfp4.quantize(np.zeros((2, 20), np.float32))
