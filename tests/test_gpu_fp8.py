@@ -242,3 +242,28 @@ def test_fp8_block_full_size_sampled_rows(kb, fp8_weights, batch, n_txt, grid, r
     assert rms(d_got - d_ref) / rms(d_ref) <= 3e-2
     assert cosine(d_got, d_ref) >= 0.999
     assert max_err_ratio(g, ref) <= FP8_MAX_ERR, max_err_ratio(g, ref)
+
+
+def test_fp8_base_model_cfg_denoise_with_stage1_cache(kb):
+    # base model (no target-level embedder) under guidance with a reference:
+    # FP8 blocks together with the text / reference stage-1 cache
+    m = ki.ModelWeights(seed=6, distilled=False, n_stage1=1, n_joint=1)
+    t = upload_model(m)
+    t["joint"] = [kb.quantize_block_e4m3(b) for b in t["joint"]]
+    t["stage1"] = {k: [kb.quantize_block_e4m3(b) for b in v] for k, v in t["stage1"].items()}
+    model = kb.KleinModel(t)
+    refs = ((3, 4),)
+    seq = kb.make_seq(2, 24, 5, 4, refs)
+    n_img, n_ref, n_total = kb.klein_seq_tokens(seq)
+    lat = ki.noise_latents(2, n_img)
+    text = ki.text_embeddings(1, 2, 24)
+    rl = ki.ref_latents(1, n_ref)
+    x = to_f32(lat)
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 2.0, seq, ws)
+    torch.cuda.synchronize()
+    ref = o.denoise(fp8.QuantizedModel(m), lat, text, rl, o.positions(24, (5, 4), refs), 3, cfg=2.0)
+    got = host(x)
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert rms(got - ref) / rms(ref) <= 3e-2, rms(got - ref) / rms(ref)
+    assert max_err_ratio(got, ref) <= FP8_MAX_ERR, max_err_ratio(got, ref)
