@@ -110,11 +110,13 @@ def quantize_block_weights(w: dict) -> dict:
 
 
 class QuantizedModel:
-    """A klein_inputs.ModelWeights whose blocks are served in rowwise FP8;
+    """A klein_inputs.ModelWeights whose blocks are served quantised (rowwise
+    FP8 by default; `quantize` may be oracle.nvfp4.quantize_block_weights);
     everything else (embedders, modulation, in/out layers) stays as is."""
 
-    def __init__(self, model):
+    def __init__(self, model, quantize=None):
         self.model = model
+        self._quantize = quantize if quantize is not None else quantize_block_weights
         self._q: dict = {}
 
     def __getattr__(self, name):
@@ -122,7 +124,7 @@ class QuantizedModel:
 
     def _quant(self, key, w):
         if key not in self._q:
-            self._q[key] = quantize_block_weights(w)
+            self._q[key] = self._quantize(w)
         return self._q[key]
 
     def stage1(self, mode: str) -> list:

@@ -36,6 +36,8 @@ import numpy as np
 
 from .fp8 import dequantize as fp8_dequantize
 from .fp8 import fake_quant as fp8_fake_quant
+from .nvfp4 import dequantize as nvfp4_dequantize
+from .nvfp4 import fake_quant_rows as nvfp4_fake_quant_rows
 
 DIM = 3072
 HEADS = 24
@@ -316,6 +318,9 @@ def block(x: np.ndarray, pos: np.ndarray, mode_of_row: np.ndarray, mod: np.ndarr
     two GEMM inputs, the normalised rows h and the concatenated
     [attention heads | SwiGLU hidden] rows, are quantised rowwise to e4m3
     and dequantised before their GEMM (oracle.fp8 states the reading).
+    NVFP4 weights (keys w_in_nv/w_out_nv, from
+    oracle.nvfp4.quantize_block_weights): the same two inputs go through NVFP4
+    with one second-level scale per row (oracle.nvfp4 states the reading).
     """
     x = np.asarray(x, F64)
     B, R, _ = x.shape
@@ -323,11 +328,16 @@ def block(x: np.ndarray, pos: np.ndarray, mode_of_row: np.ndarray, mod: np.ndarr
         rows = np.arange(R)
     rows = np.asarray(rows)
     fp8 = "w_in_q" in w
+    nv = "w_in_nv" in w
     h = modln(x, mode_of_row, mod)
     if fp8:
         h = fp8_fake_quant(h)
         w_in = fp8_dequantize(w["w_in_q"], w["w_in_s"])
         w_out = fp8_dequantize(w["w_out_q"], w["w_out_s"])
+    elif nv:
+        h = nvfp4_fake_quant_rows(h)
+        w_in = nvfp4_dequantize(*w["w_in_nv"])
+        w_out = nvfp4_dequantize(*w["w_out_nv"])
     else:
         w_in = w["w_in"]
         w_out = np.asarray(w["w_out"], F64)
@@ -343,6 +353,8 @@ def block(x: np.ndarray, pos: np.ndarray, mode_of_row: np.ndarray, mod: np.ndarr
     a_cat = np.concatenate([heads, hidden], axis=-1)
     if fp8:
         a_cat = fp8_fake_quant(a_cat)
+    elif nv:
+        a_cat = nvfp4_fake_quant_rows(a_cat)
     out = a_cat @ w_out.T          # attention output projection + MLP down-projection
     gate = mod[mode_of_row[rows], 2]
     return x[:, rows] + gate * out

@@ -19,6 +19,12 @@ Quantisation decision, in float32 (it decides integer codes):
   block scale    s_b = e4m3(amax(block) / (6 * g))     (e4m3 round-to-nearest-even, saturating)
   code               = e2m1(x / (decode(s_b) * g))     (0 where the block scale is 0)
 each operation one correctly rounded float32 step in that order.
+
+READING for the block's activations (the two GEMM inputs, made at run time):
+the second-level fp32 scale g is taken per row (token) instead of per tensor,
+so that a row's codes depend on that row alone, as in the rowwise FP8 path
+(the 16-value block scales carry the fine-grained range either way). Weights
+keep one g per matrix.
 """
 from __future__ import annotations
 
@@ -63,32 +69,52 @@ def tensor_scale(x) -> np.float32:
     return F32(amax / F32(448.0 * 6.0))
 
 
-def quantize(x, g=None):
+def quantize(x, g=None, per_row=False):
     """x [..., K] (K a multiple of 16) -> (codes uint8 [..., K], block scales
-    as e4m3 codes uint8 [..., K/16], tensor scale float32)."""
+    as e4m3 codes uint8 [..., K/16], second-level scale float32: one for the
+    tensor, or [..., 1] one per row with per_row)."""
     x32 = np.asarray(x, dtype=F64).astype(F32)
     if x32.shape[-1] % BLOCK:
         raise ValueError("the last dimension must be a multiple of 16")
-    g = tensor_scale(x32) if g is None else F32(g)
+    if per_row:
+        g = (np.max(np.abs(x32), axis=-1, keepdims=True) / F32(448.0 * 6.0)).astype(F32)
+    else:
+        g = tensor_scale(x32) if g is None else F32(g)
     blocks = x32.reshape(x32.shape[:-1] + (x32.shape[-1] // BLOCK, BLOCK))
     amax = np.max(np.abs(blocks), axis=-1)
-    if g > 0:
-        sb = e4m3_encode((amax / (F32(6.0) * g)).astype(F32))
-    else:
-        sb = np.zeros(amax.shape, np.uint8)
+    gb = np.broadcast_to(np.asarray(g, F32), amax.shape[:-1] + (1,)) if per_row else np.full((1,), g, F32)
+    ok = gb > 0
+    denom = np.where(ok, F32(6.0) * gb, F32(1.0)).astype(F32)
+    sb = np.where(ok, e4m3_encode((amax / denom).astype(F32)), np.uint8(0)).astype(np.uint8)
     sbv = e4m3_decode(sb).astype(F32)
-    step = (sbv * g).astype(F32)
+    step = (sbv * gb).astype(F32)
     safe = np.where(step > 0, step, F32(1.0)).astype(F32)
     y = np.where(step[..., None] > 0, blocks / safe[..., None], F32(0.0)).astype(F32)
     codes = e2m1_encode(y).reshape(x32.shape)
-    return codes, sb, F32(g)
+    return codes, sb, (g if per_row else F32(g))
 
 
 def dequantize(codes, sb, g) -> np.ndarray:
     c = e2m1_decode(codes)
     blocks = c.reshape(c.shape[:-1] + (c.shape[-1] // BLOCK, BLOCK))
-    return (blocks * (e4m3_decode(sb)[..., None] * F64(g))).reshape(c.shape)
+    g64 = np.asarray(g, F64)
+    scale = e4m3_decode(sb) * (g64 if g64.ndim == 0 else g64)
+    return (blocks * scale[..., None]).reshape(c.shape)
 
 
 def fake_quant(x) -> np.ndarray:
+    """Quantise with one tensor scale and dequantise."""
     return dequantize(*quantize(x))
+
+
+def fake_quant_rows(x) -> np.ndarray:
+    """Quantise with one second-level scale per row and dequantise (the
+    block's activations)."""
+    return dequantize(*quantize(x, per_row=True))
+
+
+def quantize_block_weights(w: dict) -> dict:
+    """NVFP4 copy of one block's weights (klein_inputs layout; the blocks of 16
+    run along each stored row, the GEMM's K)."""
+    return {"w_in_nv": quantize(w["w_in"]), "w_out_nv": quantize(w["w_out"]),
+            "q_norm": w["q_norm"], "k_norm": w["k_norm"]}

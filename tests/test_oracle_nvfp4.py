@@ -114,3 +114,37 @@ def test_quantised_product_error_is_the_formats():
 def test_rejects_ragged_rows():
     with pytest.raises(ValueError):
         nvfp4.quantize(np.zeros((2, 20), np.float32))
+
+
+def test_per_row_scales_make_rows_independent():
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((12, 96)) * np.exp(rng.uniform(-3, 3, (12, 1)))).astype(np.float32)
+    full = nvfp4.fake_quant_rows(x)
+    for rows in ([0], [3, 7], list(range(5, 12))):
+        np.testing.assert_array_equal(nvfp4.fake_quant_rows(x[rows]), full[rows])
+    # and each row's largest value lands on 6 x its largest block scale
+    codes, sb, g = nvfp4.quantize(x, per_row=True)
+    assert g.shape == (12, 1)
+    assert np.all(np.max(np.abs(nvfp4.e2m1_decode(codes)), axis=-1) == 6.0)
+
+
+def test_nvfp4_block_tracks_exact_block():
+    import klein_inputs as ki
+    import oracle as o
+    w = ki.block_weights(0, "joint.0")
+    wq = nvfp4.quantize_block_weights(w)
+    x = ki.tokens(1, "nvfp4blk", 1, 144)
+    pos = o.positions(80, (8, 8))
+    modes = o.mode_of_rows(80, 64, 0)
+    mod = ki.modulation_vectors(1, "nvfp4blk")
+    exact = o.block(x, pos, modes, mod, w)
+    quant = o.block(x, pos, modes, mod, wq)
+    d_e, d_q = exact - x, quant - x
+    rel = np.sqrt(np.mean((d_q - d_e) ** 2) / np.mean(d_e ** 2))
+    # four NVFP4 operands (h, W_in, the concatenated rows, W_out), each with
+    # about 0.1 relative RMS error from its 1-bit mantissa, adding incoherently:
+    # ~0.2 on the block's update; a wrong block axis or scale gives O(1)
+    assert 0.08 < rel < 0.35, rel
+    # row-subset evaluation still equals the full block (per-row activation scales)
+    rows = np.array([0, 5, 79, 80, 143])
+    np.testing.assert_allclose(o.block(x, pos, modes, mod, wq, rows=rows), quant[:, rows], rtol=0, atol=1e-12)
