@@ -350,12 +350,19 @@ def block(x: np.ndarray, pos: np.ndarray, mode_of_row: np.ndarray, mod: np.ndarr
     k = rope(rms_norm(k, w["k_norm"]), pos)
     heads = attention(q, k, v).reshape(B, len(rows), DIM)
     hidden = swiglu(hr @ w_g.T, hr @ w_u.T)
-    a_cat = np.concatenate([heads, hidden], axis=-1)
-    if fp8:
-        a_cat = fp8_fake_quant(a_cat)
-    elif nv:
-        a_cat = nvfp4_fake_quant_rows(a_cat)
-    out = a_cat @ w_out.T          # attention output projection + MLP down-projection
+    if fp8 or nv:
+        # READING (quantised files): the two down-projections take one
+        # rowwise-quantised input, the [attention heads | SwiGLU hidden] row,
+        # with a single scale across both parts.
+        a_cat = np.concatenate([heads, hidden], axis=-1)
+        a_cat = fp8_fake_quant(a_cat) if fp8 else nvfp4_fake_quant_rows(a_cat)
+        out = a_cat @ w_out.T
+    else:
+        # [blogzh] block pseudo-code: attention output (through its output
+        # projection) plus the MLP output
+        w_o = np.asarray(w_out[:, :DIM], F64)
+        w_d = np.asarray(w_out[:, DIM:], F64)
+        out = heads @ w_o.T + hidden @ w_d.T
     gate = mod[mode_of_row[rows], 2]
     return x[:, rows] + gate * out
 

@@ -396,3 +396,181 @@ def test_stage1_streams_are_isolated():
     # text stage-1 output ignores the image's latents and noise level
     np.testing.assert_array_equal(sa["txt"], sb["txt"])
     assert not np.allclose(sa["img"], sb["img"])
+
+
+# ------------------------------------------------ embedder, output layer
+
+def test_time_embed_mlp_identity_layers():
+    # With the first layer copying the 256 sinusoid values into the first 256
+    # of 3072 units and the second layer the identity, the embedder's output
+    # is SiLU of the sinusoid of 1000 sigma there and 0 elsewhere. At
+    # sigma = 0 every cosine is 1 and every sine 0: SiLU(1) = 1/(1 + 1/e).
+    w1 = np.zeros((o.DIM, o.TIME_FREQ_DIM))
+    w1[:o.TIME_FREQ_DIM] = np.eye(o.TIME_FREQ_DIM)
+    w2 = np.eye(o.DIM)
+    e = o.time_embed_mlp(w1, w2, 0.0)
+    np.testing.assert_allclose(e[:128], 1.0 / (1.0 + math.exp(-1.0)), rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(e[128:], 0.0)
+    # sigma = 0.25 -> t = 250; unit 0 is cos(250 * 1), unit 128 is sin(250 * 1)
+    e = o.time_embed_mlp(w1, w2, 0.25)
+    for u, z in ((0, math.cos(250.0)), (128, math.sin(250.0)), (1, math.cos(250.0 * 10000 ** (-1 / 128)))):
+        assert e[u] == pytest.approx(z / (1.0 + math.exp(-z)), abs=1e-12)
+    np.testing.assert_array_equal(e[256:], 0.0)
+    # the second layer acts after the activation: w2 = -I flips the sign
+    np.testing.assert_allclose(o.time_embed_mlp(w1, -w2, 0.25), -e, rtol=0, atol=1e-15)
+
+
+def test_output_layer_scale_minus_one_gives_the_shift():
+    # final (shift, scale) with scale = -1: every image row of the modulated
+    # LayerNorm equals the shift, so the velocity is W_final . shift on every
+    # row whatever the rows were; a swapped (scale, shift) order or a dropped
+    # modulation gives something else
+    rng = np.random.default_rng(21)
+    x = rng.normal(size=(2, 7, o.DIM)) * 3.0 + 1.0
+    w = ki.linear(0, "pin.final_out", o.LATENT_CH, o.DIM).astype(np.float64)
+    shift = rng.normal(size=o.DIM)
+    fm = np.stack([shift, -np.ones(o.DIM)])
+    v = o.output_layer(x, fm, w)
+    np.testing.assert_allclose(v, np.broadcast_to(w @ shift, v.shape), rtol=1e-12, atol=1e-12)
+
+
+def test_output_layer_normalises_rows():
+    # shift = scale = 0: the velocity is LayerNorm(x) . W^T, and LayerNorm
+    # removes any per-row affine change a + b x (b > 0; up to its eps of 1e-6
+    # against the variance, b >= 1 keeps that below 5e-7 relative)
+    rng = np.random.default_rng(22)
+    z = rng.normal(size=(1, 5, o.DIM))
+    w = ki.linear(0, "pin.final_out", o.LATENT_CH, o.DIM).astype(np.float64)
+    fm = np.zeros((2, o.DIM))
+    a = rng.normal(size=(1, 5, 1)) * 4.0
+    b = 1.0 + np.exp(rng.normal(size=(1, 5, 1)))
+    np.testing.assert_allclose(o.output_layer(a + b * z, fm, w), o.output_layer(z, fm, w), rtol=0, atol=2e-6)
+    zn = (z - z.mean(-1, keepdims=True)) / z.std(-1, keepdims=True)
+    np.testing.assert_allclose(o.output_layer(z, fm, w), zn @ w.T, rtol=1e-5, atol=1e-5)
+
+
+# ------------------------------------------------- transformer assembly
+
+_STACKS = {}
+
+
+def _tiny_stack(n_stage1, n_joint, distilled=True, seed=0):
+    """Seeded stacks of the model's width with few blocks; weights are
+    generated once per session and shared (treat them as read-only)."""
+    key = (n_stage1, n_joint, distilled, seed)
+    if key not in _STACKS:
+        _STACKS[key] = ki.ModelWeights(seed=seed, distilled=distilled, n_stage1=n_stage1, n_joint=n_joint)
+    return _STACKS[key]
+
+
+def test_transformer_without_blocks_is_the_output_layer_of_the_image_rows():
+    # 0 + 0 blocks: nothing mixes tokens, so the velocity is the output layer
+    # applied to the projected image latents alone; text and references
+    # change nothing
+    m = _tiny_stack(0, 0)
+    n_txt, grid, refs = 6, (3, 4), ((2, 2),)
+    pos = o.positions(n_txt, grid, refs)
+    lat = ki.noise_latents(2, 12)
+    rl = ki.ref_latents(1, 4)
+    v = o.transformer(m, lat, ki.text_embeddings(1, 2, n_txt), rl, pos, 0.7, 0.4)
+    fin = o.stage_modulations(m.misc, 0.7, 0.4)["final"]
+    expect = o.output_layer(lat.astype(np.float64) @ m.misc["img_in"].astype(np.float64).T, fin, m.misc["final_out"])
+    assert v.shape == (2, 12, o.LATENT_CH)
+    np.testing.assert_allclose(v[0], expect, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(v[1], expect, rtol=1e-12, atol=1e-12)
+    v2 = o.transformer(m, lat, ki.text_embeddings(5, 2, n_txt), None, o.positions(n_txt, grid), 0.7, 0.4)
+    np.testing.assert_allclose(v2, v, rtol=1e-12, atol=1e-12)
+
+
+def test_transformer_text_rows_are_a_set_with_their_positions():
+    # permuting the text rows together with their positions permutes the
+    # text stream (RoPE carries the order) and leaves the image velocity as
+    # it was: stage 1 is equivariant, joint attention sums over keys, and
+    # only image rows reach the output layer
+    m = _tiny_stack(1, 1, distilled=False)
+    n_txt, grid = 7, (2, 3)
+    pos = o.positions(n_txt, grid)
+    text = ki.text_embeddings(1, 1, n_txt)
+    lat = ki.noise_latents(2, 6)
+    perm = np.random.default_rng(23).permutation(n_txt)
+    pos_p = pos.copy()
+    pos_p[:n_txt] = pos[perm]
+    a = o.transformer(m, lat, text, None, pos, 0.6, None)
+    b = o.transformer(m, lat, text[:, perm], None, pos_p, 0.6, None)
+    np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-9)
+    # moving the text positions (not the rows) does change it
+    pos_q = pos.copy()
+    pos_q[:n_txt, 3] += 1.0 + np.arange(n_txt)
+    assert not np.allclose(o.transformer(m, lat, text, None, pos_q, 0.6, None), a)
+
+
+def test_transformer_references_are_context_rows_projected_by_ref_in():
+    # Without stage 1 and with the reference modulation weights set to the
+    # text ones, a reference row is a context row modulated at t = 0 like
+    # text: giving the references as references equals appending their
+    # projected latents (ref_in, not img_in) to the text with their
+    # positions. A reference projected by img_in or modulated at the image
+    # time would break the equality.
+    base = _tiny_stack(0, 2)
+    m = ki.ModelWeights(seed=0, distilled=True, n_stage1=0, n_joint=2)
+    m._blocks = base._blocks
+    m._misc = misc = dict(base.misc)
+    for st in (1, 2):
+        misc[f"mod{st}.ref"] = misc[f"mod{st}.txt"]
+    n_txt, grid, refs = 5, (2, 3), ((2, 2), (1, 3))
+    pos = o.positions(n_txt, grid, refs)
+    text = ki.text_embeddings(1, 1, n_txt)
+    lat = ki.noise_latents(2, 6)
+    rl = ki.ref_latents(1, 7)
+    a = o.transformer(m, lat, text, rl, pos, 0.8, 0.5)
+    ref_rows = rl.astype(np.float64) @ misc["ref_in"].astype(np.float64).T
+    text2 = np.concatenate([text.astype(np.float64), ref_rows[None]], axis=1)
+    pos2 = np.concatenate([pos[:n_txt], pos[n_txt + 6:], pos[n_txt:n_txt + 6]])
+    b = o.transformer(m, lat, text2, None, pos2, 0.8, 0.5)
+    np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-9)
+    # and the references do reach the image through the joint blocks only
+    s1 = _tiny_stack(1, 0)
+    c = o.transformer(s1, lat, text, rl, pos, 0.8, 0.5)
+    d = o.transformer(s1, lat, text, ki.ref_latents(4, 7), pos, 0.8, 0.5)
+    np.testing.assert_array_equal(c, d)
+    assert not np.allclose(a, o.transformer(m, lat, text, ki.ref_latents(4, 7), pos, 0.8, 0.5))
+
+
+# ----------------------------------------------------- the sampler loop
+
+@pytest.mark.parametrize("distilled", [True, False])
+def test_denoise_loop_with_exact_velocity_lands_on_x0(monkeypatch, distilled):
+    # A stand-in denoiser that returns the straight-path velocity eps - x0
+    # (for every batch item): the sampler must land on x0 exactly, for any
+    # number of steps, after visiting the shifted schedule in order; the
+    # distilled model is told sigma_next (0 on the last step), the base
+    # model is not. With guidance the two items combine by v_u + g (v_c - v_u).
+    rng = np.random.default_rng(24)
+    x0 = rng.normal(size=(9, o.LATENT_CH))
+    eps = rng.normal(size=(9, o.LATENT_CH))
+    calls = []
+
+    def stub(model, x, text, ref, pos, sigma, sigma_next, stage1_out=None):
+        calls.append((float(sigma), sigma_next))
+        np.testing.assert_allclose(x, x0 + sigma * (eps - x0), atol=1e-12)  # on the straight path
+        v = eps - x0
+        return np.stack([v, v + 7.0]) if text.shape[0] == 2 else v[None]
+
+    import oracle.klein as ok
+    monkeypatch.setattr(ok, "transformer", stub)
+    m = ki.ModelWeights(seed=0, distilled=distilled, n_stage1=0, n_joint=0)
+    m._misc = {"tt_mlp1": None} if distilled else {}   # the sampler only asks whether the target embedder exists
+    for steps in (1, 4, 16):
+        calls.clear()
+        out = o.denoise(m, eps, np.zeros((1, 3, o.DIM)), None, None, steps)
+        np.testing.assert_allclose(out, x0, atol=1e-12)
+        sig = o.sigma_schedule(steps)
+        assert [c[0] for c in calls] == pytest.approx(list(sig[:-1]), abs=0)
+        nxt = [c[1] for c in calls]
+        if distilled:
+            assert nxt == pytest.approx(list(sig[1:]), abs=0) and nxt[-1] == 0.0
+        else:
+            assert all(n is None for n in nxt)
+    # guidance 1 keeps the conditional velocity (the +7 offset is the uncond)
+    out = o.denoise(m, eps, np.zeros((2, 3, o.DIM)), None, None, 4, cfg=1.0)
+    np.testing.assert_allclose(out, x0, atol=1e-12)
