@@ -98,17 +98,20 @@ int klein_wait_probe(unsigned long long limit_ns, void* stream);
  * events on the launching stream around each kernel launch of the path and
  * tags it with its kind (index into the arrays below):
  *   0 modulated LayerNorm, 1 in-projection GEMM (QKV + MLP-in, fused
- *   epilogue), 2 attention, 3 out-projection GEMM (gated residual),
+ *   epilogue), 2 attention, 3 out-projection GEMM (gated residual) of
+ *   blocks over a whole sequence (the joint blocks);
  *   4 timestep embedding + modulation, 5 input / output projections,
  *   6 Euler update, 7 other, 8 rowwise e4m3 quantisation of the
- *   out-projection's input (FP8 blocks only).
+ *   out-projection's input (FP8 blocks only);
+ *   9, 10, 11, 12: kinds 0..3 of blocks over a row range of the sequence
+ *   (the stage-1 blocks, one stream each).
  * klein_profile_begin(max_launches) creates the events (host-side
  * resources; no device memory); klein_profile_end synchronises, writes the
  * summed milliseconds and launch counts per kind (arrays of
  * KLEIN_PROF_KINDS, either may be NULL) and releases the events. Returns
  * KLEIN_ERR_WORKSPACE if more launches happened than max_launches (those
  * were not timed). Not thread-safe; one profile at a time. */
-#define KLEIN_PROF_KINDS 9
+#define KLEIN_PROF_KINDS 13
 int klein_profile_begin(int max_launches);
 int klein_profile_end(double* ms, int* launches);
 
@@ -201,17 +204,19 @@ size_t klein_block_workspace_size(int batch, int rows);
  *   pos      device float [n_total][4] (klein_positions)
  *   mod      device float [3 modes][3 (shift, scale, gate)][3072]
  *   ws       device workspace, >= klein_block_workspace_size(batch, rows)
- * Errors: KLEIN_ERR_SHAPE if rows < 1 or the range leaves [0, n_total). */
+ * Errors: KLEIN_ERR_SHAPE if rows < 1, the range leaves [0, n_total), a
+ * stream size is negative or n_txt + n_img > n_total. */
 int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_total, int row0, int rows,
                         int n_txt, int n_img, const float* pos, const float* mod, void* ws, size_t ws_bytes,
                         void* stream);
 
 /* klein_block_forward without a workspace. The pages have no counterpart:
- * this entry point exists for callers that cannot allocate device memory,
- * for instance code being recorded into a CUDA graph under global stream
- * capture (where cudaMalloc is an error), or a plug-in whose device memory
- * is owned by a host framework's pool that it may not bypass. Same
- * arguments and results as klein_block_forward, minus ws / ws_bytes.
+ * this entry point exists for callers that cannot call cudaMalloc, such as
+ * a plug-in inside a host application that owns all device memory through
+ * its own pool and forbids allocating around it, or code on a
+ * latency-critical path where a device allocation (which may synchronise
+ * the device) is not allowed. Same arguments and results as
+ * klein_block_forward, minus ws / ws_bytes.
  *   - Scratch lives in one fixed array of this library's device memory
  *     (about 12.1 MiB), held on every GPU that loads the library until the
  *     process exits. It fits batch * round_up(rows, 128) <= 256; larger

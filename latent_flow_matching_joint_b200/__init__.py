@@ -183,7 +183,8 @@ def klein_wait_probe(limit_ns: int, stream=None):
     _check(lib.klein_wait_probe(limit_ns, _stream(stream)))
 
 
-PROF_KINDS = ("modln", "gemm_in", "attention", "gemm_out", "time_mod", "projections", "euler", "other", "quant")
+PROF_KINDS = ("modln", "gemm_in", "attention", "gemm_out", "time_mod", "projections", "euler", "other", "quant",
+              "modln_s1", "gemm_in_s1", "attention_s1", "gemm_out_s1")
 
 
 def klein_profile_begin(max_launches: int):

@@ -60,8 +60,12 @@ int num_sms() {
 // kind; klein_profile_end sums their elapsed times. Off by default: no
 // events are recorded then.
 
+// Kinds 0..3 are the four launches of a block over a whole sequence (a joint
+// block); a block over a row view of it (a stage-1 block) is recorded as
+// kind + kProfStage1 (9..12).
 enum ProfKind { kProfModln = 0, kProfGemmIn, kProfAttn, kProfGemmOut, kProfTimeMod, kProfProj, kProfEuler,
-                kProfOther, kProfQuant, kProfKinds };
+                kProfOther, kProfQuant, kProfStage1, kProfKinds = kProfStage1 + 4 };
+static_assert(kProfKinds == KLEIN_PROF_KINDS, "profiler kinds and the header's count must agree");
 
 struct Profiler {
   bool on = false;
@@ -188,8 +192,9 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   // the out-projection (in place, over the bf16 [attention | SwiGLU] rows).
   const bool f8 = wt->w_in_scale != nullptr;
   const int rows_per_tile = f8 ? 256 : kGemmRowsPerTile;
+  const int kind0 = rows == n_total ? 0 : kProfStage1;  // profiler: joint block, or a row view
   // a4: modulated LayerNorm
-  int pi = prof_begin(kProfModln, s);
+  int pi = prof_begin(kind0 + kProfModln, s);
   const int mrc = f8 ? launch_modln_e4m3(x, n_total, row0, reinterpret_cast<uint8_t*>(w.h), w.sa_h, batch, rows,
                                          n_txt, n_img, mod, 3 * kDim, s)
                      : launch_modln(x, n_total, row0, w.h, batch, rows, n_txt, n_img, mod, 3 * kDim, 0, s);
@@ -229,7 +234,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   g.rows_pad = rp;
   g.a_scale = w.sa_h;
   g.b_scale = wt->w_in_scale;
-  pi = prof_begin(kProfGemmIn, s);
+  pi = prof_begin(kind0 + kProfGemmIn, s);
   if (f8 ? launch_gemm_pair(kEpiQKV, m_h, m_win, g, s, 1) : launch_block_gemm(kEpiQKV, m_h, m_win, g, s))
     return cuda_fail("in-projection GEMM launch");
   prof_end(pi, s);
@@ -242,7 +247,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   at.out = w.a_out;
   at.out_ld = kOutK;
   at.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(128.0));
-  pi = prof_begin(kProfAttn, s);
+  pi = prof_begin(kind0 + kProfAttn, s);
   if (launch_attention(m_q, m_k, m_vt, at, s)) return cuda_fail("attention launch");
   prof_end(pi, s);
   if (f8) {
@@ -268,7 +273,7 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   o.n_img = n_img;
   o.a_scale = w.sa_o;
   o.b_scale = wt->w_out_scale;
-  pi = prof_begin(kProfGemmOut, s);
+  pi = prof_begin(kind0 + kProfGemmOut, s);
   if (f8 ? launch_gemm_pair(kEpiResid, m_aout, m_wout, o, s, 1) : launch_block_gemm(kEpiResid, m_aout, m_wout, o, s))
     return cuda_fail("out-projection GEMM launch");
   prof_end(pi, s);
@@ -498,6 +503,18 @@ static int check_block_weights(const klein_block_weights* w) {
   return KLEIN_OK;
 }
 
+// Shapes of a block call: a non-empty row range inside [0, n_total) and
+// stream sizes that fit the sequence (text rows, then image rows, the rest
+// references).
+static int check_block_rows(int batch, int n_total, int row0, int rows, int n_txt, int n_img) {
+  if (batch < 1 || n_total < 1 || rows < 1 || row0 < 0 || (long long)row0 + rows > n_total)
+    return fail(KLEIN_ERR_SHAPE, "row range [%d, %lld) outside [0, %d)", row0, (long long)row0 + rows, n_total);
+  if (n_txt < 0 || n_img < 0) return fail(KLEIN_ERR_SHAPE, "negative stream sizes");
+  if ((long long)n_txt + n_img > n_total)
+    return fail(KLEIN_ERR_SHAPE, "n_txt + n_img = %lld exceeds n_total = %d", (long long)n_txt + n_img, n_total);
+  return KLEIN_OK;
+}
+
 int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_total, int row0, int rows,
                         int n_txt, int n_img, const float* pos, const float* mod, void* ws, size_t ws_bytes,
                         void* stream) {
@@ -506,9 +523,7 @@ int klein_block_forward(const klein_block_weights* w, void* x, int batch, int n_
   if (!x || !pos || !mod || !ws) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
   if (!aligned16(x) || !aligned16(pos) || !aligned16(mod) || !aligned16(ws))
     return fail(KLEIN_ERR_ALIGN, "pointers must be 16-byte aligned");
-  if (batch < 1 || n_total < 1 || rows < 1 || row0 < 0 || row0 + rows > n_total)
-    return fail(KLEIN_ERR_SHAPE, "row range [%d, %d) outside [0, %d)", row0, row0 + rows, n_total);
-  if (n_txt < 0 || n_img < 0) return fail(KLEIN_ERR_SHAPE, "negative stream sizes");
+  if ((rc = check_block_rows(batch, n_total, row0, rows, n_txt, n_img))) return rc;
   const BlockWs bw = carve_block(ws, batch, rows);
   if (ws_bytes < bw.bytes) return fail(KLEIN_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, bw.bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

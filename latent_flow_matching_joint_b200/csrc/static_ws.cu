@@ -53,9 +53,7 @@ extern "C" int klein_block_forward_static(const klein_block_weights* w, void* x,
   if (!x || !pos || !mod) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
   if (!aligned16(x) || !aligned16(pos) || !aligned16(mod))
     return fail(KLEIN_ERR_ALIGN, "pointers must be 16-byte aligned");
-  if (batch < 1 || n_total < 1 || rows < 1 || row0 < 0 || row0 + rows > n_total)
-    return fail(KLEIN_ERR_SHAPE, "row range [%d, %d) outside [0, %d)", row0, row0 + rows, n_total);
-  if (n_txt < 0 || n_img < 0) return fail(KLEIN_ERR_SHAPE, "negative stream sizes");
+  if ((rc = check_block_rows(batch, n_total, row0, rows, n_txt, n_img))) return rc;
   const long long need_rows = (long long)batch * round_up(rows, 128);
   if (need_rows > kStaticMaxRows)
     return fail(KLEIN_ERR_WORKSPACE,

@@ -96,6 +96,13 @@ def test_argument_errors_before_any_launch(kb):
     # workspace too small
     rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1024, None)
     assert kb.STATUS[rc] == "KLEIN_ERR_WORKSPACE"
+    # stream sizes that do not fit the sequence (6 text + 5 image rows > 10)
+    for fn, extra in ((kb.lib.klein_block_forward, (256, 1 << 30)), (kb.lib.klein_block_forward_static, ())):
+        rc = fn(ctypes.byref(bw), 256, 1, 10, 0, 10, 6, 5, 256, 256, *extra, None)
+        assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
+        assert b"exceeds n_total" in kb.lib.klein_last_error()
+        rc = fn(ctypes.byref(bw), 256, 1, 10, 0, 10, -1, 5, 256, 256, *extra, None)
+        assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
     rc = kb.lib.klein_op_gemm(256, 256, 256, 10, 100, 64, None)
     assert kb.STATUS[rc] == "KLEIN_ERR_SHAPE"
     rc = kb.lib.klein_op_euler(256, 256, None, 6, ctypes.c_float(0.1), ctypes.c_float(1.0), None,
