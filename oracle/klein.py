@@ -386,7 +386,7 @@ def mode_of_rows(n_txt: int, n_img: int, n_ref: int) -> np.ndarray:
 
 def transformer(model, latents: np.ndarray, text: np.ndarray, ref_lat: np.ndarray | None,
                 pos: np.ndarray, sigma: float, sigma_next: float | None,
-                stage1_out: dict | None = None) -> np.ndarray:
+                stage1_out: dict | None = None, img_rows: np.ndarray | None = None) -> np.ndarray:
     """One denoiser call: velocity for the image tokens, [B, n_img, 128].
 
     [blog] two stages: stage 1 runs each stream (text, image, references)
@@ -402,6 +402,10 @@ def transformer(model, latents: np.ndarray, text: np.ndarray, ref_lat: np.ndarra
     layers are stacked per token and projected linearly to the model width),
     ref_lat [n_ref, 128] or None.
     If stage1_out is a dict, the stage-1 outputs per stream are stored in it.
+    If img_rows (indices into the image tokens) is given, only those rows of
+    the velocity are computed, [B, len(img_rows), 128]: the last joint block
+    evaluates just those output rows (every row still supplies keys and
+    values), as block() does for a row subset.
     """
     misc = model.misc
     text = np.asarray(text, F64)
@@ -431,9 +435,18 @@ def transformer(model, latents: np.ndarray, text: np.ndarray, ref_lat: np.ndarra
         stage1_out.update(streams)
 
     x = np.concatenate([streams[k] for k in ("txt", "img", "ref") if k in streams], axis=1)
-    for w in model.joint():
-        x = block(x, pos, modes, mods[2], w)
-    return output_layer(x[:, n_txt:n_txt + n_img], mods["final"], misc["final_out"])
+    joint = model.joint()
+    if img_rows is None:
+        for w in joint:
+            x = block(x, pos, modes, mods[2], w)
+        return output_layer(x[:, n_txt:n_txt + n_img], mods["final"], misc["final_out"])
+    out_rows = n_txt + np.asarray(img_rows)
+    for i, w in enumerate(joint):
+        last = i == len(joint) - 1
+        x = block(x, pos, modes, mods[2], w, rows=out_rows if last else None)
+    if not joint:
+        x = x[:, out_rows]
+    return output_layer(x, mods["final"], misc["final_out"])
 
 
 def denoise(model, noise: np.ndarray, text: np.ndarray, ref_lat: np.ndarray | None,

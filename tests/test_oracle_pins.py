@@ -574,3 +574,20 @@ def test_denoise_loop_with_exact_velocity_lands_on_x0(monkeypatch, distilled):
     # guidance 1 keeps the conditional velocity (the +7 offset is the uncond)
     out = o.denoise(m, eps, np.zeros((2, 3, o.DIM)), None, None, 4, cfg=1.0)
     np.testing.assert_allclose(out, x0, atol=1e-12)
+
+
+def test_transformer_image_row_subset():
+    # the velocity of a subset of image rows equals those rows of the full
+    # velocity (the last joint block evaluates only the subset's outputs)
+    m = _tiny_stack(1, 1, distilled=False)
+    n_txt, grid = 7, (2, 3)
+    pos = o.positions(n_txt, grid)
+    text = ki.text_embeddings(1, 1, n_txt)
+    lat = ki.noise_latents(2, 6)
+    full = o.transformer(m, lat, text, None, pos, 0.6, None)
+    rows = np.array([0, 3, 5])
+    sub = o.transformer(m, lat, text, None, pos, 0.6, None, img_rows=rows)
+    np.testing.assert_allclose(sub, full[:, rows], rtol=1e-12, atol=1e-12)
+    m0 = _tiny_stack(0, 0)
+    np.testing.assert_allclose(o.transformer(m0, lat, text, None, pos, 0.6, 0.2, img_rows=rows),
+                               o.transformer(m0, lat, text, None, pos, 0.6, 0.2)[:, rows], rtol=1e-12, atol=1e-12)
