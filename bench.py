@@ -10,7 +10,7 @@ same size (1.3916 TFLOP) is timed alone in the same run, before the denoise,
 and reported as `joint_block`.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload t2i|edit|cfg2048|edit3|t2i4k|block|memory] [--precision bf16|fp8]
+                    [--workload t2i|edit|cfg2048|edit3|t2i4k|block|memory] [--precision bf16|fp8|nvfp4]
                     [--no-cpu-baseline]
 """
 from __future__ import annotations
@@ -30,7 +30,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "joint-block TFLOP/s & denoise steps/s at 1024² (frac of B200 BF16 peak)"
 DIM, MLP, LAT = 3072, 9216, 128
-DTYPES = {"bf16": "bf16", "fp8": "e4m3 rowwise (block GEMMs), bf16 elsewhere"}
+DTYPES = {"bf16": "bf16", "fp8": "e4m3 rowwise (block GEMMs), bf16 elsewhere",
+          "nvfp4": "nvfp4: e2m1 + e4m3 block scales per 16 (block GEMMs), bf16 elsewhere"}
 
 WORKLOADS = {
     # name: (batch, n_txt, img grid, refs, steps, cfg, distilled, description)
@@ -51,14 +52,17 @@ WORKLOADS = {
 # Rowwise FP8 (e4m3) runs the two block GEMMs at the e4m3 tensor rate: the
 # measured bf16 peak times the nominal dense ratio (4.5 / 2.25 PFLOP/s).
 FP8_OVER_BF16 = 2.0
+# NVFP4 (block-scaled e2m1) runs at the nominal dense fp4 / bf16 ratio (9 / 2.25 PFLOP/s).
+FP4_OVER_BF16 = 4.0
+PEAK_RATIO = {"bf16": 1.0, "fp8": FP8_OVER_BF16, "nvfp4": FP4_OVER_BF16}
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one bf16 in-projection GEMM
 # launch (gemm_pair_kernel<2, 0>) over 512 + 4096 rows, the launch shape of
 # every joint block of the 1024x1024 denoise, from an ncu capture of
 # `bench.py --workload block` (one joint block; its summary is kept with the
-# other kernel profiles). None until captured on the current kernel; must be
-# re-captured (or set to None) whenever that kernel changes.
-GEMM_IN_TRAFFIC_BYTES = None
+# other kernel profiles). Must be re-captured (or set to None) whenever that
+# kernel changes.
+GEMM_IN_TRAFFIC_BYTES = 356.29e6
 
 
 def load_peaks():
@@ -291,11 +295,12 @@ def random_block(g, dev):
 def to_precision(t, precision):
     """Rowwise FP8 copies of every block of a model dict (the bf16 block
     weights are dropped); other weights stay bf16."""
-    if precision != "fp8":
+    if precision == "bf16":
         return t
     import latent_flow_matching_joint_b200 as kb
-    t["stage1"] = {m: [kb.quantize_block_e4m3(b) for b in bl] for m, bl in t["stage1"].items()}
-    t["joint"] = [kb.quantize_block_e4m3(b) for b in t["joint"]]
+    q = kb.quantize_block_e4m3 if precision == "fp8" else kb.quantize_block_nvfp4
+    t["stage1"] = {m: [q(b) for b in bl] for m, bl in t["stage1"].items()}
+    t["joint"] = [q(b) for b in t["joint"]]
     return t
 
 
@@ -330,6 +335,8 @@ def run_block_only(args):
     bw = random_block(g, dev)
     if args.precision == "fp8":
         bw = kb.quantize_block_e4m3(bw)
+    elif args.precision == "nvfp4":
+        bw = kb.quantize_block_nvfp4(bw)
     x = torch.randn(1, 4608, DIM, generator=g, device=dev)
     pos = torch.empty(4608, 4, device=dev)
     kb.klein_positions(kb.make_seq(1, 512, 64, 64), pos)
@@ -475,7 +482,7 @@ def run_ours(args):
     n_img, n_ref, n_total = kb.klein_seq_tokens(seq)
     model_t = to_precision(random_model(dev, distilled, bool(refs), seed=0), args.precision)
     model = kb.KleinModel(model_t)
-    fp8 = args.precision == "fp8"
+    fp8 = args.precision != "bf16"   # a quantised block (rowwise FP8 or NVFP4)
     g = torch.Generator(device=dev).manual_seed(1 + rank)
     noise = torch.randn(n_img, LAT, generator=g, device=dev)
     text = torch.randn(batch, n_txt, DIM, generator=g, device=dev).to(torch.bfloat16)
@@ -576,12 +583,12 @@ def run_ours(args):
     gi_flops = gi_n * gi_rows * 2.0 * DIM * (3 * DIM + 2 * MLP)
     gi_avg_ms = gi_ms / max(gi_n, 1)
     achieved = gi_flops / (gi_ms / 1e3) / 1e12 if gi_ms > 0 else 0.0
-    gi_peak = peaks["bf16_sustained"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    gi_peak = peaks["bf16_sustained"] * PEAK_RATIO[args.precision]
     all_in_ms = gi_ms + prof["gemm_in_s1"][0]
     all_in_flops = gemm_in_rows_per_denoise(batch, n_txt, n_img, n_ref, steps, distilled) * args.steps * 2.0 * DIM * (
         3 * DIM + 2 * MLP)
     roofline = {"kernel": f"gemm_in of the joint blocks (fused QKV + MLP-in, tcgen05"
-                          f"{', e4m3' if fp8 else ''}; {gi_rows} rows x 3072 -> 27648 per launch)",
+                          f"{', ' + args.precision if fp8 else ''}; {gi_rows} rows x 3072 -> 27648 per launch)",
                 "bound": "tensor", "achieved": achieved, "peak": gi_peak, "unit": "TFLOP/s",
                 "frac": achieved / gi_peak,
                 "traffic": GEMM_IN_TRAFFIC_BYTES if (gi_rows == 4608 and not fp8) else None,
@@ -591,7 +598,8 @@ def run_ours(args):
                 "all_in_projection_launches_tflops": all_in_flops / (all_in_ms / 1e3) / 1e12 if all_in_ms else None,
                 "timing": "CUDA events around each launch on its stream, second pass of the same K denoises",
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"
-                + (" x 2 (nominal e4m3 / bf16 dense ratio)" if fp8 else "")}
+                + ({"bf16": "", "fp8": " x 2 (nominal e4m3 / bf16 dense ratio)",
+                    "nvfp4": " x 4 (nominal fp4 / bf16 dense ratio)"}[args.precision])}
 
     # ---- end to end through the public API with host buffers
     noise_h = noise.cpu().pin_memory()
@@ -632,9 +640,12 @@ def run_ours(args):
         "config": {"workload": desc, "global_batch": world * batch, "seq_len": n_total, "parallelism": f"replicas x{world}",
                    "euler_steps_per_bench_step": steps, "cfg": cfg, "distilled": distilled,
                    "precision": args.precision,
-                   "l2": "working set > L2 (" + ("5.6" if fp8 else "11") + " GB of weights streamed per Euler step)",
+                   "l2": "working set > L2 (" + {"bf16": "11", "fp8": "5.6", "nvfp4": "3.0"}[args.precision]
+                         + " GB of weights streamed per Euler step)",
                    "weights": "random init N(0, 1/fan_in), bf16" + (
-                       "; block weights rowwise e4m3 (one scale per output row)" if fp8 else ""),
+                       {"bf16": "", "fp8": "; block weights rowwise e4m3 (one scale per output row)",
+                        "nvfp4": "; block weights NVFP4 (e2m1, e4m3 scale per 16 values, fp32 per matrix)"}[
+                           args.precision]),
                    "inputs": "N(0,1) noise and text embeddings"},
         # the method's FLOPs per step (every batch item's streams counted)
         "tflops_per_gpu": f_step * steps * args.steps / (ms / 1e3) / 1e12,

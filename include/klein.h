@@ -165,7 +165,19 @@ int klein_positions(const klein_seq* seq, float* pos, void* stream);
  *          them. The block quantises its two GEMM inputs (the modulated
  *          LayerNorm rows, and the [attention | SwiGLU] rows) the same way
  *          per token and runs both GEMMs on e4m3 tensor cores with fp32
- *          accumulation; everything else is as in the bf16 block. */
+ *          accumulation; everything else is as in the bf16 block.
+ *   w_in_sf, w_out_sf  NULL unless the block is NVFP4 (the transformer's
+ *          nvfp4 file, same blog section; NVFP4 runs on Blackwell tensor
+ *          cores, "How to Run FLUX 3 Image Klein Locally"). Both set: w_in
+ *          and w_out hold e2m1 codes as klein_quantize_nvfp4 writes them
+ *          (w_in [27648][1536] bytes in the in-projection order of
+ *          KLEIN_NVFP4_IN_PROJ, w_out [3072][6144]), w_in_sf / w_out_sf their
+ *          block scales, and w_in_scale / w_out_scale each point to ONE float,
+ *          the matrix's second-level scale. The block quantises its two GEMM
+ *          inputs to NVFP4 per token (one second-level scale per row) and runs
+ *          both GEMMs on the block-scaled fp4 tensor cores with fp32
+ *          accumulation; attention and everything else stay as in the bf16
+ *          block. */
 typedef struct {
   const void* w_in;
   const void* w_out;
@@ -173,7 +185,37 @@ typedef struct {
   const float* k_norm;
   const float* w_in_scale;
   const float* w_out_scale;
+  const void* w_in_sf;
+  const void* w_out_sf;
 } klein_block_weights;
+
+/* NVFP4 quantisation of a bf16 matrix src [rows][cols] (row pitch cols):
+ * e2m1 values (1 sign, 2 exponent bits with bias 1, 1 mantissa bit;
+ * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one e4m3 scale per 16 consecutive
+ * values of a row, and fp32 second-level scales. All decisions in fp32, each
+ * step one correctly rounded operation: g = amax / 2688 (0 if all zero);
+ * block scale s = e4m3_rn_satfinite(amax_block / (6 g)); code =
+ * e2m1_rn_satfinite(x / (s g)), 0 where s g = 0.
+ *   mode   KLEIN_NVFP4_MATRIX: one g for the matrix (amax over all of it),
+ *          written to g[0]; KLEIN_NVFP4_ROWS: one g per row (g[rows]);
+ *          KLEIN_NVFP4_IN_PROJ: as MATRIX for a block's w_in [27648][3072],
+ *          with the output rows in the NVFP4 in-projection's order: q, k, v
+ *          rows (0..9215) as they are, then for each 64-unit chunk c of the
+ *          SwiGLU hidden its gate rows 64c..64c+63 and its up rows 64c..64c+63.
+ *   codes  device [rows][cols / 2] bytes; value 2i in the low 4 bits of byte i
+ *   sf     device, round_up(rows, P) * cols / 16 bytes, P = 256 in ROWS mode
+ *          and 128 otherwise: 512-byte atoms, atom (R, C) for rows
+ *          128R..128R+127 and columns 64C..64C+63 at byte (R * cols / 64 + C)
+ *          * 512, the scale of row r, block b (0..3 in the atom's 64 columns)
+ *          at (r % 32) * 16 + ((r % 128) / 32) * 4 + b; padding rows get 0.
+ *          This is the order in which the tensor core reads block scales.
+ * cols a multiple of 64, at most 12288; codes must not overlap src.
+ * Errors: KLEIN_ERR_SHAPE, KLEIN_ERR_ALIGN, KLEIN_ERR_INVALID_ARG. */
+#define KLEIN_NVFP4_MATRIX 0
+#define KLEIN_NVFP4_ROWS 1
+#define KLEIN_NVFP4_IN_PROJ 2
+int klein_quantize_nvfp4(const void* src, long long rows, int cols, int mode, void* codes, void* sf, float* g,
+                         void* stream);
 
 /* Rowwise e4m3 quantisation of a bf16 matrix src [rows][cols] (row pitch
  * cols): codes [rows][cols] bytes, scale [rows] float. Per row, in fp32:
@@ -296,10 +338,14 @@ int klein_stack_forward(const klein_model* m, const float* latents, const void* 
  * (sigma_next - sigma) * v. cfg > 1 needs seq->batch == 2 (text = cond then
  * uncond) and uses v = v_u + cfg (v_c - v_u); otherwise seq->batch == 1.
  *   latents  device float [n_img][128]: in = noise, out = the final latents
- *   x0_out   device float [n_img][128] or NULL: the last step's x0 preview */
+ *   x0_out   device float or NULL: the x0 preview x0 = x - sigma v of a step,
+ *            taken before that step's update ([guide] "The denoise loop";
+ *            [blogzh] Modular Diffusers preview block, a preview after every
+ *            denoiser call): with x0_every_step = 0, [n_img][128] receives the
+ *            last step's; otherwise [steps][n_img][128] receives every step's */
 int klein_denoise(const klein_model* m, float* latents, const void* text, const float* refs, int steps,
-                  float cfg, float shift, const klein_seq* seq, float* x0_out, void* ws, size_t ws_bytes,
-                  void* stream);
+                  float cfg, float shift, const klein_seq* seq, float* x0_out, int x0_every_step, void* ws,
+                  size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ single ops
  * The kernels of the path, exposed one by one for parity tests and the
@@ -341,6 +387,22 @@ int klein_op_gemm_e4m3(const void* a, const float* a_scale, const void* b, const
  * the fp32 normalised rows). Per-stream modes as in klein_block_forward. */
 int klein_op_modln_e4m3(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
                         const float* mod, long long mod_stride, void* codes, float* scale, void* stream);
+
+/* klein_op_modln with the output quantised to NVFP4 as the NVFP4 block's
+ * first step does (KLEIN_NVFP4_ROWS rule on the fp32 normalised rows):
+ * codes [batch][rows][1536] bytes, sf per batch item over round_up(rows, 256)
+ * rows (the layout of klein_quantize_nvfp4; batch item b at b *
+ * round_up(rows, 256) * 192 bytes), g [batch][rows]. */
+int klein_op_modln_nvfp4(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
+                         const float* mod, long long mod_stride, void* codes, void* sf, float* g, void* stream);
+
+/* C[m][n] (float) = a_g[row] * (*b_g) * sum_k (A code * A block scale)
+ * (B code * B block scale) on the block-scaled fp4 tensor cores of the NVFP4
+ * block. A: codes [m][k/2] with scales over round_up(m, 256) rows and a_g
+ * [m] (klein_quantize_nvfp4 in ROWS mode); B: codes [n][k/2] with scales and
+ * one b_g (MATRIX mode). M >= 1, N a multiple of 128, K a multiple of 256. */
+int klein_op_gemm_nvfp4(const void* a, const void* a_sf, const float* a_g, const void* b, const void* b_sf,
+                        const float* b_g, float* c, int m, int n, int k, void* stream);
 
 /* Softmax attention per (batch, head) over `rows` rows, scale 1/sqrt(128),
  * no mask. q, k: bf16 [batch][24][rows_pad][128]; vt: bf16

@@ -49,7 +49,10 @@ class KleinSeq(Structure):
 
 class KleinBlockWeights(Structure):
     _fields_ = [("w_in", c_void_p), ("w_out", c_void_p), ("q_norm", c_void_p), ("k_norm", c_void_p),
-                ("w_in_scale", c_void_p), ("w_out_scale", c_void_p)]
+                ("w_in_scale", c_void_p), ("w_out_scale", c_void_p), ("w_in_sf", c_void_p), ("w_out_sf", c_void_p)]
+
+
+NVFP4_MATRIX, NVFP4_ROWS, NVFP4_IN_PROJ = 0, 1, 2
 
 
 class KleinModelDesc(Structure):
@@ -84,7 +87,7 @@ _SIGS = {
     "klein_stack_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float, POINTER(KleinSeq),
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "klein_denoise": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float, c_float, POINTER(KleinSeq),
-                              c_void_p, c_void_p, c_size_t, c_void_p]),
+                              c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "klein_op_modln": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_longlong, c_int,
                                c_void_p, c_void_p]),
     "klein_op_rope_table": (c_int, [c_void_p, c_int, c_float, c_void_p, c_void_p]),
@@ -99,6 +102,11 @@ _SIGS = {
     "klein_quantize_rowwise_e4m3": (c_int, [c_void_p, c_longlong, c_int, c_void_p, c_void_p, c_void_p]),
     "klein_op_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_longlong,
                                    c_void_p]),
+    "klein_quantize_nvfp4": (c_int, [c_void_p, c_longlong, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "klein_op_modln_nvfp4": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_longlong,
+                                     c_void_p, c_void_p, c_void_p, c_void_p]),
+    "klein_op_gemm_nvfp4": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                    c_int, c_void_p]),
     "klein_op_time_mod": (c_int, [c_void_p, c_float, c_float, c_int, c_void_p, c_void_p, c_void_p, c_size_t,
                                   c_void_p]),
 }
@@ -215,11 +223,13 @@ def klein_positions(seq: KleinSeq, pos, stream=None):
 
 def block_weights(w: dict) -> KleinBlockWeights:
     """KleinBlockWeights from a dict of CUDA tensors w_in, w_out, q_norm, k_norm
-    (+ w_in_scale, w_out_scale for a rowwise FP8 block, see quantize_block_e4m3)."""
-    si, so = w.get("w_in_scale"), w.get("w_out_scale")
-    return KleinBlockWeights(w["w_in"].data_ptr(), w["w_out"].data_ptr(), w["q_norm"].data_ptr(),
-                             w["k_norm"].data_ptr(), si.data_ptr() if si is not None else None,
-                             so.data_ptr() if so is not None else None)
+    (+ w_in_scale, w_out_scale for a rowwise FP8 block, see quantize_block_e4m3;
+    + w_in_sf, w_out_sf for an NVFP4 block, see quantize_block_nvfp4)."""
+    def p(name):
+        t = w.get(name)
+        return t.data_ptr() if t is not None else None
+    return KleinBlockWeights(p("w_in"), p("w_out"), p("q_norm"), p("k_norm"), p("w_in_scale"), p("w_out_scale"),
+                             p("w_in_sf"), p("w_out_sf"))
 
 
 def klein_quantize_rowwise_e4m3(src, codes, scale, stream=None):
@@ -240,6 +250,49 @@ def quantize_block_e4m3(w: dict, stream=None) -> dict:
         klein_quantize_rowwise_e4m3(src, codes, scale, stream)
         out[name], out[name + "_scale"] = codes, scale
     return out
+
+
+def nvfp4_scale_bytes(rows: int, cols: int, mode: int) -> int:
+    """Bytes of the block-scale atoms klein_quantize_nvfp4 writes."""
+    pad = 256 if mode == NVFP4_ROWS else 128
+    return (rows + pad - 1) // pad * pad * cols // 16
+
+
+def klein_quantize_nvfp4(src, mode: int, stream=None):
+    """NVFP4 codes (uint8 [rows, cols/2]), block scales (uint8 atoms) and
+    second-level scales (float32 [1] or [rows]) of a bf16 [rows, cols] CUDA
+    tensor (new device tensors)."""
+    import torch
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=src.device)
+    sf = torch.empty(nvfp4_scale_bytes(rows, cols, mode), dtype=torch.uint8, device=src.device)
+    g = torch.empty(rows if mode == NVFP4_ROWS else 4, dtype=torch.float32, device=src.device)
+    _check(lib.klein_quantize_nvfp4(_ptr(src), rows, cols, mode, _ptr(codes), _ptr(sf), _ptr(g), _stream(stream)))
+    return codes, sf, g
+
+
+def quantize_block_nvfp4(w: dict, stream=None) -> dict:
+    """An NVFP4 copy of one block's bf16 weights (new device tensors); w_in
+    in the in-projection's NVFP4 row order."""
+    out = {"q_norm": w["q_norm"], "k_norm": w["k_norm"]}
+    for name, mode in (("w_in", NVFP4_IN_PROJ), ("w_out", NVFP4_MATRIX)):
+        codes, sf, g = klein_quantize_nvfp4(w[name], mode, stream)
+        out[name], out[name + "_sf"], out[name + "_scale"] = codes, sf, g
+    return out
+
+
+def klein_op_modln_nvfp4(x, row0: int, rows: int, n_txt: int, n_img: int, mod, codes, sf, g, stream=None):
+    batch, n_total = x.shape[0], x.shape[1]
+    stride = mod.shape[-2] * mod.shape[-1]
+    _check(lib.klein_op_modln_nvfp4(_ptr(x), batch, n_total, row0, rows, n_txt, n_img, _ptr(mod), stride, _ptr(codes),
+                                    _ptr(sf), _ptr(g), _stream(stream)))
+
+
+def klein_op_gemm_nvfp4(a, a_sf, a_g, b, b_sf, b_g, c, stream=None):
+    m, kh = a.shape
+    n = b.shape[0]
+    _check(lib.klein_op_gemm_nvfp4(_ptr(a), _ptr(a_sf), _ptr(a_g), _ptr(b), _ptr(b_sf), _ptr(b_g), _ptr(c), m, n,
+                                   2 * kh, _stream(stream)))
 
 
 def klein_block_forward(w: dict, x, n_txt: int, n_img: int, pos, mod, ws, row0: int = 0, rows: int | None = None,
@@ -317,10 +370,10 @@ def klein_stack_forward(model: KleinModel, latents, text, refs, sigma: float, si
 
 
 def klein_denoise(model: KleinModel, latents, text, refs, steps: int, cfg: float, seq: KleinSeq, ws,
-                  shift: float = 6.93, x0_out=None, stream=None):
+                  shift: float = 6.93, x0_out=None, x0_every_step: bool = False, stream=None):
     _check(lib.klein_denoise(model.handle, _ptr(latents), _ptr(text), _ptr(refs), steps, cfg, shift,
-                             ctypes.byref(seq), _ptr(x0_out), _ptr(ws), ws.numel() * ws.element_size(),
-                             _stream(stream)))
+                             ctypes.byref(seq), _ptr(x0_out), int(x0_every_step), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def klein_op_modln(x, row0: int, rows: int, n_txt: int, n_img: int, mod, h, single_mode: bool = False,

@@ -7,7 +7,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libklein.so")
-SOURCES = ["klein_all.cu", "kernels_mem.cu", "gemm.cu", "attention.cu", "klein_capi.cu", "static_ws.cu", "common.cuh",
+SOURCES = ["klein_all.cu", "kernels_mem.cu", "gemm.cu", "attention.cu", "nvfp4.cu", "klein_capi.cu", "static_ws.cu", "common.cuh",
            "internal.h", os.path.join("..", "..", "include", "klein.h")]
 
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

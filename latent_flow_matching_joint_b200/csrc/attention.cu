@@ -21,7 +21,10 @@
 //               the bound keeps P <= 256. Final 1/l normalisation and bf16
 //               store into the out-projection's A operand.
 // Tensor memory (512 columns): tile t owns S_t (128 fp32 columns, P_t in its
-// first 64 as packed bf16) and O_t (128 fp32 columns).
+// first 64 as packed bf16) and O_t (128 fp32 columns). P stays in tensor
+// memory: written to shared memory instead, its stores and the MMA's reads of
+// it add about 96 KB of shared-memory traffic per key tile on top of the
+// operands, more than the shared-memory bandwidth leaves room for.
 // Keys past the end of the view are zero-filled by TMA and masked to -inf.
 #include <math.h>
 
@@ -54,6 +57,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_empty = bars + 5;  // [2]
   uint64_t* s_full = bars + 7;    // [2 tiles]: scores ready (phase j), final output ready (phase nkv)
   uint64_t* p_full = bars + 9;    // [2 tiles][2 halves of the keys]
+  uint64_t* drain = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5;
@@ -74,6 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[2 * s], 128);
       mbar_init(&p_full[2 * s + 1], 128);
     }
+    mbar_init(drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_q);
     tma_prefetch_desc(&map_k);
@@ -88,6 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+  pdl_trigger();
+  pdl_wait();  // q, k, v^T and the output are touched only after the previous kernel completes
 
   if (warp == 0) {
     if (lane == 0) {
@@ -96,17 +103,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(smem + kOffQ + t * kTileBytes, &map_q, q_full, 0, q_row0 + 128 * t, bh);
         tma_load_3d(smem + kOffQ + t * kTileBytes + kTileBytes / 2, &map_q, q_full, 64, q_row0 + 128 * t, bh);
       }
+      StageLog klog, vlog;
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, 0x201)) break;
         uint8_t* kd = smem + kOffK + st * kTileBytes;
         uint8_t* vd = smem + kOffV + st * kTileBytes;
         mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+        klog.armed(st, (j >> 1) & 1);
         tma_load_3d(kd, &map_k, &k_full[st], 0, j * 128, bh);
         tma_load_3d(kd + kTileBytes / 2, &map_k, &k_full[st], 64, j * 128, bh);
         mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+        vlog.armed(st, (j >> 1) & 1);
         tma_load_3d(vd, &map_vt, &v_full[st], j * 128, 0, bh);
         tma_load_3d(vd + kTileBytes / 2, &map_vt, &v_full[st], j * 128 + 64, 0, bh);
+      }
+      // no TMA write may land in shared memory after the CTA exits
+      if (mbar_wait(q_full, 0, 0x209)) {
+        klog.drain(k_full, 2, 0x209);
+        vlog.drain(v_full, 2, 0x209);
       }
     }
   } else if (warp == 1) {
@@ -155,6 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // every MMA issued here has completed before TMEM is freed
+      umma_commit(drain);
+      mbar_wait(drain, 0, 0x20a);
     }
   } else {
     const int t = (warp - 2) >> 2;         // query tile of this warpgroup
@@ -265,8 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mvt, const AttnArgs& a,
-                     cudaStream_t s) {
+int launch_attention(const AttnArgs& a, cudaStream_t s) {
   static bool configured[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0) return -1;
@@ -276,10 +293,18 @@ int launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     configured[dev] = true;
   }
   if (a.rows <= 0 || a.batch <= 0) return 0;
-  dim3 grid((a.rows + 255) / 256, a.heads, a.batch);
-  attn_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mvt, a);
+  CUtensorMap mq, mk, mvt;
+  const uint64_t bh = (uint64_t)a.batch * a.heads, rp = a.rows_pad;
+  if (make_map_3d(&mq, a.q, kHeadDim, a.rows, bh, kHeadDim * 2, rp * kHeadDim * 2, 64, 128) ||
+      make_map_3d(&mk, a.k, kHeadDim, a.rows, bh, kHeadDim * 2, rp * kHeadDim * 2, 64, 128) ||
+      make_map_3d(&mvt, a.vt, a.rows, kHeadDim, bh, rp * 2, rp * kHeadDim * 2, 64, 128))
+    return -2;
+  const cudaError_t e = launch_kernel(attn_kernel, dim3((a.rows + 255) / 256, a.heads, a.batch), dim3(kThreads), kSmem,
+                                      s, 1, mq, mk, mvt, a);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
+
+
 
 }  // namespace klein

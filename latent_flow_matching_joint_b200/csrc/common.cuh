@@ -5,8 +5,12 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
+
+#include <utility>
 
 namespace klein {
 
@@ -108,6 +112,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels of the path are launched so that each may start (barrier set-up,
+// TMEM allocation, descriptor prefetch, CTA scheduling) while the kernel
+// before it on the stream finishes. Every such kernel lets its successor
+// launch as soon as it starts (pdl_trigger: the successor's CTAs then take
+// SMs that this grid's last wave frees) and, before its first access to
+// global memory that an earlier kernel writes or reads, waits for the
+// previous kernel to complete with its writes visible (pdl_wait). Because
+// every kernel waits, a kernel never completes before its predecessor, so
+// the ordering is transitive along the stream. Without the launch attribute
+// both instructions do nothing.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -154,6 +172,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
     }
   }
 }
+
+// Non-blocking test of a phase with cluster-scope acquire (for barriers that
+// threads of the other CTA of a pair arrive on).
+__device__ __forceinline__ bool mbar_test_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Stages of a TMA ring whose full barrier this thread armed, and the phase
+// of each last arming. drain() waits (bounded) for those phases, so that a
+// producer that stops early (a wait gave up) leaves no TMA write in flight
+// into shared memory when its CTA exits. On the normal path every phase has
+// completed already and drain() returns at once. A stage's last armed phase
+// is the only pending one, so waiting on its parity cannot alias a later one.
+struct StageLog {
+  uint32_t armed_mask = 0, phase_bits = 0;
+  __device__ __forceinline__ void armed(int stage, uint32_t phase) {
+    armed_mask |= 1u << stage;
+    phase_bits = (phase_bits & ~(1u << stage)) | ((phase & 1u) << stage);
+  }
+  __device__ __forceinline__ void drain(uint64_t* full, int stages, unsigned site) const {
+    for (int s = 0; s < stages; ++s)
+      if ((armed_mask >> s) & 1u)
+        if (!mbar_wait(&full[s], (phase_bits >> s) & 1u, site)) return;
+  }
+};
 
 // ------------------------------------------------------------------ TMA
 
@@ -449,6 +500,16 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
       : "memory");
 }
 
+// Per-warpgroup register budget (every warp of the warpgroup executes it).
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -474,6 +535,47 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t* r) {
 // Row -> stream mode by global row index within one batch item.
 __device__ __forceinline__ int mode_of_row(int row, int n_txt, int n_img) {
   return row < n_txt ? 0 : (row < n_txt + n_img ? 1 : 2);
+}
+
+// ------------------------------------------------------------------ host: launches
+
+// Whether kernels are launched with programmatic dependent launch (on unless
+// the environment sets KLEIN_PDL=0; read once per process).
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("KLEIN_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Launches `kernel` on `s` with programmatic dependent launch (see
+// pdl_wait) and, for cluster_x > 1, clusters of cluster_x CTAs along x.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace klein

@@ -253,7 +253,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* empty = full + Cfg::kStages;
   uint64_t* acc_full = empty + Cfg::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 128);
     }
+    mbar_init(drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
@@ -279,6 +281,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // operands and outputs are touched only after the previous kernel completes
 
   const int m_tiles = g.batch * g.m_tiles_per_b;
   const int total = m_tiles * g.n_tiles;
@@ -288,6 +292,7 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      StageLog log;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
         const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
@@ -306,6 +311,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < g.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, 0x101)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::kStage);
+          log.armed(stage, phase);
           uint8_t* sa = smem + stage * Cfg::kStage;
           uint8_t* sb = sa + Cfg::kStageA;
           tma_load_3d(sa, &map_a, &full[stage], kb * 64, row0, b);
@@ -315,6 +321,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!ok) break;
       }
+      log.drain(full, Cfg::kStages, 0x105);  // no TMA write may land after the CTA exits
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -342,6 +349,9 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         umma_commit(&acc_full[acc]);
       }
+      // every MMA issued here has completed before TMEM is freed
+      umma_commit(drain);
+      mbar_wait(drain, 0, 0x106);
     }
   } else {
     const int quarter = warp & 3;
@@ -390,9 +400,9 @@ static int launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmAr
   const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
   if (total <= 0) return 0;
   const int grid = total < num_sms() ? total : num_sms();
-  gemm_kernel<BN, EPI><<<grid, Cfg::kThreads, Cfg::kSmem, s>>>(ma, mb, g);
+  const cudaError_t e = launch_kernel(gemm_kernel<BN, EPI>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, s, 1, ma, mb, g);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ---- CTA-pair variant: 256 x 256 output tiles per cluster of 2 CTAs.
@@ -432,7 +442,8 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
   uint64_t* empty = full + Cfg::kStages;
   uint64_t* acc_full = empty + Cfg::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -448,6 +459,7 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 2 * 32 * Cfg::kEpiWarps);
     }
+    mbar_init(drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
@@ -460,6 +472,8 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
   cluster_sync();  // barrier initialisation and the TMEM allocation are visible pair-wide
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // operands and outputs are touched only after the previous kernel completes
 
   const int m_tiles = g.batch * g.m_tiles_per_b;
   const int total = m_tiles * g.n_tiles;
@@ -472,6 +486,7 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      StageLog log;
       for (int tile = pair; tile < total; tile += npairs) {
         const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
         const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
@@ -487,7 +502,10 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
         bool ok = true;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, 0x111)) { ok = false; break; }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStage);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStage);
+            log.armed(stage, phase);
+          }
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* sa = smem + stage * Cfg::kStage;
           tma_load_3d_pair(sa, &map_a, bar, kb * kBlockK, row0, b);
@@ -496,6 +514,11 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
         }
         if (!ok) break;
       }
+      // The even CTA's full barriers count the bytes of both CTAs' loads:
+      // once every phase it armed is complete, no TMA write of the pair is
+      // still in flight (the cluster barrier below keeps the odd CTA alive
+      // until then).
+      if (leader) log.drain(full, Cfg::kStages, 0x115);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -525,6 +548,9 @@ __global__ void __launch_bounds__(PairCfg::kThreads, 1)
         if (!ok) break;
         umma_commit_pair(&acc_full[acc], 0x3);
       }
+      // every pair MMA issued here has completed before either CTA frees its TMEM
+      umma_commit_pair(drain, 0x1);
+      mbar_wait(drain, 0, 0x116);
     }
   } else {
     const int quarter = warp & 3;
@@ -590,8 +616,8 @@ static int launch_pair_one(const CUtensorMap& ma, const CUtensorMap& mb, const G
   const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
   if (total <= 0) return 0;
   const int pairs = total < max_pairs ? total : max_pairs;
-  cfg.gridDim = dim3(2 * pairs);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI, F8>, ma, mb, g);
+  const cudaError_t e =
+      launch_kernel(gemm_pair_kernel<EPI, F8>, dim3(2 * pairs), dim3(Cfg::kThreads), Cfg::kSmem, s, 2, ma, mb, g);
   note_launch();
   return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }

@@ -19,6 +19,9 @@ int make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t out
 // 3-D bf16 tensor map over [d2][d1][d0] with byte strides s1 (d1) and s2 (d2).
 int make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                 uint64_t s2, uint32_t box0, uint32_t box1, int bytes1 = 0);
+// 2-D map of 32-bit words [outer][inner], no swizzle (dense boxes).
+int make_map_2d_u32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer);
 
 // ------------------------------------------------------------------ GEMM
 
@@ -61,6 +64,8 @@ struct GemmArgs {
   // e4m3 operands (launch_gemm_pair with e4m3 = 1): acc * a_scale[b * rows + r] * b_scale[B row]
   const float* a_scale;
   const float* b_scale;
+  // NVFP4 operands (launch_gemm_nvfp4): acc * a_scale[b * rows + r] * (*b_g)
+  const float* b_g;
 };
 
 // C[M,N] = A[M,K] * B[N,K]^T with epilogue `epi`; bn = 128 or 256.
@@ -74,17 +79,40 @@ int launch_gemm_pair(int epi, const CUtensorMap& map_a, const CUtensorMap& map_b
 int launch_gemm(int bn, int epi, const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& args,
                 cudaStream_t stream);
 
+// NVFP4 GEMM on CTA pairs (256 x 128 tiles; args.m_tiles_per_b counts 256-row
+// tiles, n_tiles 128-column tiles, k_blocks 256-value K blocks): A codes
+// [batch][rows][K/2] with scale atoms over round_up(rows, 256) rows per batch
+// item, B codes [n_rows_b][K/2] with scale atoms (n_rows_b a multiple of
+// 128); epi is kEpiF32, kEpiQKV (tile n < 72: head n % 24 of q, k, v; else
+// 64 SwiGLU hidden units, B rows 64 gate then 64 up) or kEpiResid.
+int launch_gemm_nvfp4(int epi, const void* a, long long a_ld, const void* a_sf, const void* b, const void* b_sf,
+                      const GemmArgs& args, int n_rows_b, cudaStream_t stream);
+// NVFP4 quantisation of `batch` bf16 matrices [rows][cols] (see nvfp4.cu);
+// g_matrix: one scale for the whole (single) matrix, computed here;
+// otherwise one per row into g_rows. in_proj_order: the in-projection
+// weights' rows in the NVFP4 GEMM's tile order.
+int launch_quantize_nvfp4(const __nv_bfloat16* src, long long src_ld, int in_proj_order, uint8_t* dst,
+                          long long dst_ld, uint8_t* sf, float* g_rows, float* g_matrix, int batch, int rows,
+                          int rows_pad, int cols, cudaStream_t stream);
+int launch_modln_nvfp4(const float* x, long long x_bstride, int x_row0, uint8_t* codes, uint8_t* sf, float* g_rows,
+                       int batch, int rows, int n_txt, int n_img, const float* mod, long long mod_stride,
+                       cudaStream_t stream);
+
 // ------------------------------------------------------------------ attention
 
 struct AttnArgs {
   int batch, heads, rows, rows_pad;
-  __nv_bfloat16* out;   // [batch][rows][out_ld], head h at columns h*128..
+  const __nv_bfloat16* q;   // [batch][heads][rows_pad][128]
+  const __nv_bfloat16* k;   // [batch][heads][rows_pad][128]
+  const __nv_bfloat16* vt;  // [batch][heads][128][rows_pad]
+  __nv_bfloat16* out;       // [batch][rows][out_ld], head h at columns h*128..
   long long out_ld;
-  float scale_log2;     // log2(e) / sqrt(128)
+  float scale_log2;         // log2(e) / sqrt(128)
 };
 
-int launch_attention(const CUtensorMap& map_q, const CUtensorMap& map_k, const CUtensorMap& map_vt,
-                     const AttnArgs& args, cudaStream_t stream);
+// Builds the operand tensor maps and launches the attention kernel.
+// Returns 0, -1 on a launch error, -2 if a tensor map cannot be encoded.
+int launch_attention(const AttnArgs& args, cudaStream_t stream);
 
 // ------------------------------------------------------------------ memory-bound kernels
 

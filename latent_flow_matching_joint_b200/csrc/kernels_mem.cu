@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256, 2) modln_kernel(const float* __restrict__
                                                     int rows, int n_txt, int n_img,
                                                     const float* __restrict__ mod, long long mod_stride,
                                                     int single_mode) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= batch * rows) return;
@@ -68,10 +70,10 @@ int launch_modln(const float* x, long long x_bstride, int x_row0, __nv_bfloat16*
   const long long warps = (long long)batch * rows;
   if (warps <= 0) return 0;
   const int blocks = (int)((warps + 7) / 8);
-  modln_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, h, batch, rows, n_txt, n_img, mod, mod_stride,
+  const cudaError_t le = launch_kernel(modln_kernel, dim3(blocks), dim3(256), 0, s, 1, x, x_bstride, x_row0, h, batch, rows, n_txt, n_img, mod, mod_stride,
                                       single_mode);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ---- rowwise e4m3 quantisation (the transformer's rowwise FP8 weights,
@@ -94,6 +96,8 @@ __global__ void __launch_bounds__(256, 1) modln_e4m3_kernel(const float* __restr
                                                          float* __restrict__ scale, int batch, int rows,
                                                          int n_txt, int n_img, const float* __restrict__ mod,
                                                          long long mod_stride) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= batch * rows) return;
@@ -155,10 +159,10 @@ int launch_modln_e4m3(const float* x, long long x_bstride, int x_row0, uint8_t* 
   const long long warps = (long long)batch * rows;
   if (warps <= 0) return 0;
   const int blocks = (int)((warps + 7) / 8);
-  modln_e4m3_kernel<<<blocks, 256, 0, s>>>(x, x_bstride, x_row0, reinterpret_cast<uint32_t*>(codes), scale, batch,
+  const cudaError_t le = launch_kernel(modln_e4m3_kernel, dim3(blocks), dim3(256), 0, s, 1, x, x_bstride, x_row0, reinterpret_cast<uint32_t*>(codes), scale, batch,
                                            rows, n_txt, n_img, mod, mod_stride);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // One CTA of 256 threads per row; 8 bf16 per thread per chunk, at most 6
@@ -169,6 +173,8 @@ constexpr int kQuantMaxChunks = 6;
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* src, long long src_ld,
                                                             uint8_t* dst, long long dst_ld,
                                                             float* __restrict__ scale, int cols) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[8];
   const long long row = blockIdx.x;
   const int nchunks = cols >> 3;
@@ -212,9 +218,9 @@ int launch_quantize_rows(const __nv_bfloat16* src, long long src_ld, uint8_t* ds
                          long long rows, int cols, cudaStream_t s) {
   if (rows <= 0) return 0;
   if (cols <= 0 || cols % 8 || cols > 256 * 8 * kQuantMaxChunks || rows > 0x7fffffffLL) return -2;
-  quantize_rows_kernel<<<(unsigned)rows, 256, 0, s>>>(src, src_ld, dst, dst_ld, scale, cols);
+  const cudaError_t le = launch_kernel(quantize_rows_kernel, dim3((unsigned)rows), dim3(256), 0, s, 1, src, src_ld, dst, dst_ld, scale, cols);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // bf16 rows -> fp32 rows of the residual stream: src [batch][rows][3072]
@@ -222,6 +228,8 @@ int launch_quantize_rows(const __nv_bfloat16* src, long long src_ld, uint8_t* ds
 // of each batch item (batch stride dst_bstride rows).
 __global__ void rows_to_f32_kernel(const uint4* __restrict__ src, long long src_bstride, float4* __restrict__ dst,
                                    long long dst_bstride, int dst_row0, int rows, long long total) {
+  pdl_trigger();
+  pdl_wait();
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total) return;
   constexpr int kPerRow = kDim / 8;
@@ -240,11 +248,11 @@ int launch_rows_to_f32(const __nv_bfloat16* src, long long src_bstride, float* d
                        int dst_row0, int batch, int rows, cudaStream_t s) {
   const long long total = (long long)batch * rows * (kDim / 8);
   if (total <= 0) return 0;
-  rows_to_f32_kernel<<<(int)((total + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(src), src_bstride,
+  const cudaError_t le = launch_kernel(rows_to_f32_kernel, dim3((int)((total + 255) / 256)), dim3(256), 0, s, 1, reinterpret_cast<const uint4*>(src), src_bstride,
                                                                   reinterpret_cast<float4*>(dst), dst_bstride,
                                                                   dst_row0, rows, total);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ RoPE
@@ -254,6 +262,8 @@ int launch_rows_to_f32(const __nv_bfloat16* src, long long src_bstride, float* d
 
 __global__ void rope_table_kernel(const float* __restrict__ pos, float2* __restrict__ table, int rows,
                                   double theta) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= rows * kPairs) return;
   const int r = idx / kPairs;
@@ -270,15 +280,17 @@ __global__ void rope_table_kernel(const float* __restrict__ pos, float2* __restr
 int launch_rope_table(const float* pos, float2* table, int rows, float theta, cudaStream_t s) {
   const int n = rows * kPairs;
   if (n <= 0) return 0;
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(pos, table, rows, static_cast<double>(theta));
+  const cudaError_t le = launch_kernel(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, s, 1, pos, table, rows, static_cast<double>(theta));
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // Standalone rotation of [rows][heads][128] bf16 (the same arithmetic as the
 // in-projection epilogue). One thread per 8 elements (4 pairs).
 __global__ void rope_apply_kernel(const uint4* __restrict__ in, uint4* __restrict__ out,
                                   const float2* __restrict__ table, int rows, int heads) {
+  pdl_trigger();
+  pdl_wait();
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long total = (long long)rows * heads * (kHeadDim / 8);
   if (idx >= total) return;
@@ -302,10 +314,10 @@ int launch_rope_apply(const __nv_bfloat16* in, __nv_bfloat16* out, const float2*
   const long long total = (long long)rows * heads * (kHeadDim / 8);
   if (total <= 0) return 0;
   const int blocks = (int)((total + 255) / 256);
-  rope_apply_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out),
+  const cudaError_t le = launch_kernel(rope_apply_kernel, dim3(blocks), dim3(256), 0, s, 1, reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out),
                                            table, rows, heads);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ positions
@@ -321,6 +333,8 @@ struct RefDims {
 
 __global__ void positions_kernel(float* __restrict__ pos, int n_txt, int img_h, int img_w, RefDims refs,
                                  int total) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= total) return;
   float t = 0.f, hh = 0.f, ww = 0.f, l = 0.f;
@@ -358,9 +372,9 @@ int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, co
     total += ref_h[k] * ref_w[k];
   }
   if (total <= 0) return 0;
-  positions_kernel<<<(total + 255) / 256, 256, 0, s>>>(pos, n_txt, img_h, img_w, rd, total);
+  const cudaError_t le = launch_kernel(positions_kernel, dim3((total + 255) / 256), dim3(256), 0, s, 1, pos, n_txt, img_h, img_w, rd, total);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ Euler + CFG
@@ -370,6 +384,8 @@ int launch_positions(float* pos, int n_txt, int img_h, int img_w, int n_refs, co
 
 __global__ void euler_kernel(float4* __restrict__ x, const float4* __restrict__ vc, const float4* __restrict__ vu,
                              long long n4, float dsigma, float g, float4* __restrict__ x0, float sigma) {
+  pdl_trigger();
+  pdl_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   float4 v = __ldcs(vc + i);
@@ -392,14 +408,16 @@ int launch_euler(float* x, const float* vc, const float* vu, long long n, float 
   if (n <= 0) return 0;
   const long long n4 = n / 4;
   const int blocks = (int)((n4 + 255) / 256);
-  euler_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(vc),
+  const cudaError_t le = launch_kernel(euler_kernel, dim3(blocks), dim3(256), 0, s, 1, reinterpret_cast<float4*>(x), reinterpret_cast<const float4*>(vc),
                                       reinterpret_cast<const float4*>(vu), n4, dsigma, g,
                                       reinterpret_cast<float4*>(x0), sigma);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 __global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, long long n4) {
+  pdl_trigger();
+  pdl_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   const float4 v = in[i];
@@ -409,10 +427,10 @@ __global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict_
 int launch_to_bf16(const float* in, __nv_bfloat16* out, long long n, cudaStream_t s) {
   if (n <= 0) return 0;
   const long long n4 = n / 4;
-  to_bf16_kernel<<<(int)((n4 + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(in),
+  const cudaError_t le = launch_kernel(to_bf16_kernel, dim3((int)((n4 + 255) / 256)), dim3(256), 0, s, 1, reinterpret_cast<const float4*>(in),
                                                          reinterpret_cast<uint2*>(out), n4);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ GEMV
@@ -425,6 +443,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restri
                                                    const float* __restrict__ x, int n_vec, long long x_stride,
                                                    float* __restrict__ y, long long y_stride, int act_silu,
                                                    const float* __restrict__ add) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float xs[];  // [n_vec][k]
   for (int i = threadIdx.x; i < n_vec * k; i += blockDim.x) {
     const int vv = i / k;
@@ -474,9 +494,9 @@ int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_
       return -1;
     configured[dev] = true;
   }
-  gemv_kernel<<<(n_out + 7) / 8, 256, smem, s>>>(w, n_out, k, x, n_vec, x_stride, y, y_stride, act_silu, add);
+  const cudaError_t le = launch_kernel(gemv_kernel, dim3((n_out + 7) / 8), dim3(256), smem, s, 1, w, n_out, k, x, n_vec, x_stride, y, y_stride, act_silu, add);
   note_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+  return (le == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ time embedding + modulation
@@ -487,6 +507,8 @@ int launch_gemv(const __nv_bfloat16* w, int n_out, int k, const float* x, int n_
 // W * SiLU(e) split into (shift, scale, gate).
 
 __global__ void sinusoid_kernel(float* __restrict__ out, float t0, float t1, float t2) {
+  pdl_trigger();
+  pdl_wait();
   const int i = threadIdx.x;  // 0..127
   const int v = blockIdx.x;   // 0..2
   const double t = 1000.0 * static_cast<double>(v == 0 ? t0 : (v == 1 ? t1 : t2));
@@ -504,9 +526,9 @@ int launch_time_mod(const TimeModArgs& a, cudaStream_t s) {
   float* e = h1 + 2 * kDim;
   float* tg1 = e + 2 * kDim;
   float* tg = tg1 + kDim;
-  sinusoid_kernel<<<3, 128, 0, s>>>(sin_v, a.sigma, 0.0f, a.sigma_next);
+  const cudaError_t le = launch_kernel(sinusoid_kernel, dim3(3), dim3(128), 0, s, 1, sin_v, a.sigma, 0.0f, a.sigma_next);
   note_launch();
-  if (cudaGetLastError() != cudaSuccess) return -1;
+  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return -1;
   const float* add = nullptr;
   if (a.tt_mlp1) {
     if (launch_gemv(a.tt_mlp1, kDim, 256, sin_v + 2 * 256, 1, 256, tg1, kDim, 0, nullptr, s)) return -1;

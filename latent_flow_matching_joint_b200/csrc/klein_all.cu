@@ -4,5 +4,6 @@
 #include "kernels_mem.cu"
 #include "gemm.cu"
 #include "attention.cu"
+#include "nvfp4.cu"
 #include "klein_capi.cu"
 #include "static_ws.cu"

@@ -117,6 +117,19 @@ int make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t out
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+int make_map_2d_u32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  if (get_encode()) return -1;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
 int make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                 uint64_t s2, uint32_t box0, uint32_t box1, int bytes1) {
   if (get_encode()) return -1;
@@ -140,7 +153,8 @@ static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t
 struct BlockWs {
   __nv_bfloat16 *h, *q, *k, *vt, *a_out;
   float2* rope;
-  float *sa_h, *sa_o;  // FP8 blocks: per-row scales of the two GEMM inputs
+  float *sa_h, *sa_o;  // FP8 / NVFP4 blocks: per-row scales of the two GEMM inputs
+  uint8_t *sf_h, *sf_o;  // NVFP4 blocks: block scales of the two GEMM inputs (atoms over round_up(rows, 256) rows)
   int rows_pad;
   size_t bytes;
 };
@@ -163,6 +177,9 @@ static BlockWs carve_block(void* base, int batch, int rows) {
   w.rope = reinterpret_cast<float2*>(take((size_t)rows * kPairs * sizeof(float2)));
   w.sa_h = reinterpret_cast<float*>(take((size_t)batch * rows * sizeof(float)));
   w.sa_o = reinterpret_cast<float*>(take((size_t)batch * rows * sizeof(float)));
+  const size_t rp256 = (size_t)round_up(rows, 256);
+  w.sf_h = reinterpret_cast<uint8_t*>(take((size_t)batch * rp256 * (kDim / 16)));
+  w.sf_o = reinterpret_cast<uint8_t*>(take((size_t)batch * rp256 * (kOutK / 16)));
   w.bytes = off;
   return w;
 }
@@ -183,9 +200,87 @@ static int launch_block_gemm(int epi, const CUtensorMap& ma, const CUtensorMap& 
 
 // One block over rows [row0, row0+rows) of x. `rope` holds the view's table
 // (row 0 = global row row0). Workspace `w` is carved for (batch, >= rows).
+// NVFP4 block (weights with block scales): modLN quantised to NVFP4 ->
+// NVFP4 in-projection -> attention -> in-place NVFP4 quantisation of the
+// [attention | SwiGLU] rows -> NVFP4 out-projection.
+static int block_impl_nvfp4(const klein_block_weights* wt, float* x, int batch, int n_total, int row0, int rows,
+                            int n_txt, int n_img, const float2* rope, const float* mod, const BlockWs& w,
+                            cudaStream_t s) {
+  const int rp = round_up(rows, 128);
+  const int kind0 = rows == n_total ? 0 : kProfStage1;
+  int pi = prof_begin(kind0 + kProfModln, s);
+  if (launch_modln_nvfp4(x, n_total, row0, reinterpret_cast<uint8_t*>(w.h), w.sf_h, w.sa_h, batch, rows, n_txt,
+                         n_img, mod, 3 * kDim, s))
+    return cuda_fail("modln launch");
+  prof_end(pi, s);
+  GemmArgs g{};
+  g.batch = batch;
+  g.rows = rows;
+  g.m_tiles_per_b = (rows + 255) / 256;
+  g.n_tiles = (kInCols) / 128;
+  g.k_blocks = kDim / 256;
+  g.q = w.q;
+  g.k = w.k;
+  g.vt = w.vt;
+  g.a_out = w.a_out;
+  g.q_norm = wt->q_norm;
+  g.k_norm = wt->k_norm;
+  g.rope = rope;
+  g.rows_pad = rp;
+  g.a_scale = w.sa_h;
+  g.b_g = wt->w_in_scale;
+  pi = prof_begin(kind0 + kProfGemmIn, s);
+  int rc = launch_gemm_nvfp4(kEpiQKV, w.h, kDim / 2, w.sf_h, wt->w_in, wt->w_in_sf, g, kInCols, s);
+  if (rc == -2) return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  if (rc) return cuda_fail("in-projection GEMM launch");
+  prof_end(pi, s);
+  AttnArgs at{};
+  at.batch = batch;
+  at.heads = kHeads;
+  at.rows = rows;
+  at.rows_pad = rp;
+  at.q = w.q;
+  at.k = w.k;
+  at.vt = w.vt;
+  at.out = w.a_out;
+  at.out_ld = kOutK;
+  at.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(128.0));
+  pi = prof_begin(kind0 + kProfAttn, s);
+  if (launch_attention(at, s)) return cuda_fail("attention launch");
+  prof_end(pi, s);
+  pi = prof_begin(kProfQuant, s);
+  if (launch_quantize_nvfp4(w.a_out, kOutK, 0, reinterpret_cast<uint8_t*>(w.a_out), (long long)kOutK * 2, w.sf_o,
+                            w.sa_o, nullptr, batch, rows, round_up(rows, 256), kOutK, s))
+    return cuda_fail("quantisation launch");
+  prof_end(pi, s);
+  GemmArgs o{};
+  o.batch = batch;
+  o.rows = rows;
+  o.m_tiles_per_b = (rows + 255) / 256;
+  o.n_tiles = kDim / 128;
+  o.k_blocks = kOutK / 256;
+  o.n_fastest = 1;
+  o.x = x;
+  o.x_bstride = n_total;
+  o.x_row0 = row0;
+  o.mod = mod;
+  o.n_txt = n_txt;
+  o.n_img = n_img;
+  o.a_scale = w.sa_o;
+  o.b_g = wt->w_out_scale;
+  pi = prof_begin(kind0 + kProfGemmOut, s);
+  // the codes sit at the start of each bf16 [attention | SwiGLU] row (pitch 24576 bytes)
+  rc = launch_gemm_nvfp4(kEpiResid, w.a_out, (long long)kOutK * 2, w.sf_o, wt->w_out, wt->w_out_sf, o, kDim, s);
+  if (rc == -2) return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  if (rc) return cuda_fail("out-projection GEMM launch");
+  prof_end(pi, s);
+  return KLEIN_OK;
+}
+
 static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_total, int row0, int rows,
                       int n_txt, int n_img, const float2* rope, const float* mod, const BlockWs& w,
                       cudaStream_t s) {
+  if (wt->w_in_sf) return block_impl_nvfp4(wt, x, batch, n_total, row0, rows, n_txt, n_img, rope, mod, w, s);
   const int rp = round_up(rows, 128);
   // Rowwise FP8 blocks: both GEMMs on e4m3 codes (CTA pairs); the GEMM
   // inputs are quantised per row where they are made (modLN) or just before
@@ -201,17 +296,11 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   if (mrc) return cuda_fail("modln launch");
   prof_end(pi, s);
   // a5: fused in-projection
-  CUtensorMap m_h, m_win, m_q, m_k, m_vt, m_aout, m_wout;
+  CUtensorMap m_h, m_win, m_aout, m_wout;
   const int eb = f8 ? 1 : 2;                // operand bytes per element
   const uint32_t bk = f8 ? 128 : 64;        // elements per 128-byte K box
   if (make_map_3d(&m_h, w.h, kDim, rows, batch, (uint64_t)kDim * eb, (uint64_t)rows * kDim * eb, bk, 128, f8) ||
       make_map_2d(&m_win, wt->w_in, kDim, kInCols, (uint64_t)kDim * eb, bk, 128, f8) ||
-      make_map_3d(&m_q, w.q, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rp * kHeadDim * 2,
-                  64, 128) ||
-      make_map_3d(&m_k, w.k, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rp * kHeadDim * 2,
-                  64, 128) ||
-      make_map_3d(&m_vt, w.vt, rows, kHeadDim, (uint64_t)batch * kHeads, (uint64_t)rp * 2,
-                  (uint64_t)rp * kHeadDim * 2, 64, 128) ||
       // the out-projection's A keeps the bf16 row pitch: FP8 codes are written in place
       make_map_3d(&m_aout, w.a_out, kOutK, rows, batch, (uint64_t)kOutK * 2, (uint64_t)rows * kOutK * 2, bk, 128,
                   f8) ||
@@ -244,11 +333,14 @@ static int block_impl(const klein_block_weights* wt, float* x, int batch, int n_
   at.heads = kHeads;
   at.rows = rows;
   at.rows_pad = rp;
+  at.q = w.q;
+  at.k = w.k;
+  at.vt = w.vt;
   at.out = w.a_out;
   at.out_ld = kOutK;
   at.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(128.0));
   pi = prof_begin(kind0 + kProfAttn, s);
-  if (launch_attention(m_q, m_k, m_vt, at, s)) return cuda_fail("attention launch");
+  if (launch_attention(at, s)) return cuda_fail("attention launch");
   prof_end(pi, s);
   if (f8) {
     pi = prof_begin(kProfQuant, s);
@@ -354,7 +446,7 @@ extern "C" {
 
 const char* klein_last_error(void) { return g_msg; }
 
-int klein_version(void) { return 102; }
+int klein_version(void) { return 103; }
 
 long long klein_launch_count(void) { return g_launches; }
 
@@ -498,7 +590,12 @@ static int check_block_weights(const klein_block_weights* w) {
     return fail(KLEIN_ERR_ALIGN, "block weights must be 16-byte aligned");
   if ((w->w_in_scale == nullptr) != (w->w_out_scale == nullptr))
     return fail(KLEIN_ERR_INVALID_ARG, "FP8 block weights need both w_in_scale and w_out_scale");
-  if ((w->w_in_scale && !aligned16(w->w_in_scale)) || (w->w_out_scale && !aligned16(w->w_out_scale)))
+  if ((w->w_in_sf == nullptr) != (w->w_out_sf == nullptr))
+    return fail(KLEIN_ERR_INVALID_ARG, "NVFP4 block weights need both w_in_sf and w_out_sf");
+  if (w->w_in_sf && !w->w_in_scale)
+    return fail(KLEIN_ERR_INVALID_ARG, "NVFP4 block weights need their second-level scales (w_in_scale, w_out_scale)");
+  if ((w->w_in_scale && !aligned16(w->w_in_scale)) || (w->w_out_scale && !aligned16(w->w_out_scale)) ||
+      (w->w_in_sf && !aligned16(w->w_in_sf)) || (w->w_out_sf && !aligned16(w->w_out_sf)))
     return fail(KLEIN_ERR_ALIGN, "weight scales must be 16-byte aligned");
   return KLEIN_OK;
 }
@@ -783,7 +880,8 @@ int klein_stack_forward(const klein_model* m, const float* latents, const void* 
 }
 
 int klein_denoise(const klein_model* m, float* latents, const void* text, const float* refs, int steps, float cfg,
-                  float shift, const klein_seq* seq, float* x0_out, void* ws, size_t ws_bytes, void* stream) {
+                  float shift, const klein_seq* seq, float* x0_out, int x0_every_step, void* ws, size_t ws_bytes,
+                  void* stream) {
   int ni = 0, nr = 0, nt = 0;
   int rc = check_stack_args(m, latents, text, refs, seq, ws, ws_bytes, &ni, &nr, &nt);
   if (rc) return rc;
@@ -822,9 +920,10 @@ int klein_denoise(const klein_model* m, float* latents, const void* text, const 
                     s);
     if (rc) break;
     const float dsig = static_cast<float>(static_cast<double>(sig[i + 1]) - static_cast<double>(sig[i]));
+    // x0 preview of this step (before its update): every step's, or the last one's
+    float* x0 = !x0_out ? nullptr : (x0_every_step ? x0_out + (size_t)i * n : (i == steps - 1 ? x0_out : nullptr));
     const int pi = prof_begin(kProfEuler, s);
-    if (launch_euler(latents, w.v, guided ? w.v + n : nullptr, n, dsig, cfg, (i == steps - 1) ? x0_out : nullptr,
-                     sig[i], s))
+    if (launch_euler(latents, w.v, guided ? w.v + n : nullptr, n, dsig, cfg, x0, sig[i], s))
       rc = cuda_fail("euler launch");
     prof_end(pi, s);
   }
@@ -955,6 +1054,67 @@ int klein_op_modln_e4m3(const void* x, int batch, int n_total, int row0, int row
   return KLEIN_OK;
 }
 
+int klein_quantize_nvfp4(const void* src, long long rows, int cols, int mode, void* codes, void* sf, float* g,
+                         void* stream) {
+  if (!src || !codes || !sf || !g) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(src) || !aligned16(codes) || !aligned16(sf) || !aligned16(g))
+    return fail(KLEIN_ERR_ALIGN, "unaligned pointer");
+  if (mode < KLEIN_NVFP4_MATRIX || mode > KLEIN_NVFP4_IN_PROJ) return fail(KLEIN_ERR_INVALID_ARG, "bad mode");
+  if (rows < 1 || rows > (1 << 30) || cols < 64 || (cols % 64) != 0 || cols > kOutK)
+    return fail(KLEIN_ERR_SHAPE, "need rows >= 1 and cols a multiple of 64 in [64, 12288]");
+  if (mode == KLEIN_NVFP4_IN_PROJ && (rows != kInCols || cols != kDim))
+    return fail(KLEIN_ERR_SHAPE, "the in-projection order needs a [27648][3072] matrix");
+  const char* s0 = static_cast<const char*>(src);
+  const char* c0 = static_cast<const char*>(codes);
+  if (c0 < s0 + rows * cols * 2 && s0 < c0 + rows * cols / 2) return fail(KLEIN_ERR_INVALID_ARG, "codes overlap src");
+  const bool per_row = mode == KLEIN_NVFP4_ROWS;
+  const int rows_pad = round_up(static_cast<int>(rows), per_row ? 256 : 128);
+  if (launch_quantize_nvfp4(static_cast<const __nv_bfloat16*>(src), cols, mode == KLEIN_NVFP4_IN_PROJ,
+                            static_cast<uint8_t*>(codes), cols / 2, static_cast<uint8_t*>(sf), per_row ? g : nullptr,
+                            per_row ? nullptr : g, 1, static_cast<int>(rows), rows_pad, cols,
+                            static_cast<cudaStream_t>(stream)))
+    return cuda_fail("quantisation launch");
+  return KLEIN_OK;
+}
+
+int klein_op_modln_nvfp4(const void* x, int batch, int n_total, int row0, int rows, int n_txt, int n_img,
+                         const float* mod, long long mod_stride, void* codes, void* sf, float* g, void* stream) {
+  if (!x || !mod || !codes || !sf || !g) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(x) || !aligned16(mod) || !aligned16(codes) || !aligned16(sf) || !aligned16(g) || (mod_stride % 4) != 0)
+    return fail(KLEIN_ERR_ALIGN, "pointers must be 16-byte aligned, mod_stride a multiple of 4");
+  if (batch < 1 || rows < 1 || row0 < 0 || row0 + rows > n_total) return fail(KLEIN_ERR_SHAPE, "bad row range");
+  if (launch_modln_nvfp4(static_cast<const float*>(x), n_total, row0, static_cast<uint8_t*>(codes),
+                         static_cast<uint8_t*>(sf), g, batch, rows, n_txt, n_img, mod, mod_stride,
+                         static_cast<cudaStream_t>(stream)))
+    return cuda_fail("modln launch");
+  return KLEIN_OK;
+}
+
+int klein_op_gemm_nvfp4(const void* a, const void* a_sf, const float* a_g, const void* b, const void* b_sf,
+                        const float* b_g, float* c, int m, int n, int k, void* stream) {
+  if (!a || !a_sf || !a_g || !b || !b_sf || !b_g || !c) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(a) || !aligned16(a_sf) || !aligned16(a_g) || !aligned16(b) || !aligned16(b_sf) || !aligned16(b_g) ||
+      !aligned16(c))
+    return fail(KLEIN_ERR_ALIGN, "unaligned pointer");
+  if (m < 1 || n < 128 || (n % 128) != 0 || k < 256 || (k % 256) != 0)
+    return fail(KLEIN_ERR_SHAPE, "need M >= 1, N a multiple of 128, K a multiple of 256");
+  GemmArgs g{};
+  g.batch = 1;
+  g.rows = m;
+  g.m_tiles_per_b = (m + 255) / 256;
+  g.n_tiles = n / 128;
+  g.k_blocks = k / 256;
+  g.out = c;
+  g.out_ld = n;
+  g.out_bstride = m;
+  g.a_scale = a_g;
+  g.b_g = b_g;
+  const int rc = launch_gemm_nvfp4(kEpiF32, a, k / 2, a_sf, b, b_sf, g, n, static_cast<cudaStream_t>(stream));
+  if (rc == -2) return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  if (rc) return cuda_fail("gemm launch");
+  return KLEIN_OK;
+}
+
 int klein_op_attention(const void* q, const void* k, const void* vt, int batch, int rows, int rows_pad, void* out,
                        long long out_ld, void* stream) {
   if (!q || !k || !vt || !out) return fail(KLEIN_ERR_INVALID_ARG, "NULL pointer argument");
@@ -962,23 +1122,20 @@ int klein_op_attention(const void* q, const void* k, const void* vt, int batch, 
     return fail(KLEIN_ERR_ALIGN, "unaligned pointer or out_ld");
   if (batch < 1 || rows < 1 || rows_pad < rows || (rows_pad % 8) != 0 || out_ld < kDim)
     return fail(KLEIN_ERR_SHAPE, "bad attention shape");
-  CUtensorMap mq, mk, mv;
-  if (make_map_3d(&mq, q, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rows_pad * kHeadDim * 2,
-                  64, 128) ||
-      make_map_3d(&mk, k, kHeadDim, rows, (uint64_t)batch * kHeads, kHeadDim * 2, (uint64_t)rows_pad * kHeadDim * 2,
-                  64, 128) ||
-      make_map_3d(&mv, vt, rows, kHeadDim, (uint64_t)batch * kHeads, (uint64_t)rows_pad * 2,
-                  (uint64_t)rows_pad * kHeadDim * 2, 64, 128))
-    return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   AttnArgs at{};
   at.batch = batch;
   at.heads = kHeads;
   at.rows = rows;
   at.rows_pad = rows_pad;
+  at.q = static_cast<const __nv_bfloat16*>(q);
+  at.k = static_cast<const __nv_bfloat16*>(k);
+  at.vt = static_cast<const __nv_bfloat16*>(vt);
   at.out = static_cast<__nv_bfloat16*>(out);
   at.out_ld = out_ld;
   at.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(128.0));
-  if (launch_attention(mq, mk, mv, at, static_cast<cudaStream_t>(stream))) return cuda_fail("attention launch");
+  const int arc = launch_attention(at, static_cast<cudaStream_t>(stream));
+  if (arc == -2) return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  if (arc) return cuda_fail("attention launch");
   return KLEIN_OK;
 }
 

@@ -12,13 +12,16 @@ namespace klein {
 
 // Largest batch * round_up(rows, 128) the fixed scratch can hold.
 constexpr int kStaticMaxRows = 256;
-// Bytes of carve_block(1, kStaticMaxRows): h, q, k, v^T, attention|SwiGLU
-// operand, RoPE table, the two per-row FP8 scale vectors (every region is a
-// multiple of 256 bytes).
+// Bytes of carve_block(batch, rows) for every batch * round_up(rows, 128) <=
+// kStaticMaxRows: h, q, k, v^T, attention|SwiGLU operand, RoPE table, the two
+// per-row scale vectors, and the NVFP4 block scales of the two GEMM inputs,
+// laid out per batch item over round_up(rows, 256) rows (at most 2 *
+// kStaticMaxRows rows in all). Every region is a multiple of 256 bytes.
 constexpr size_t kStaticWsBytes = (size_t)kStaticMaxRows * kDim * 2 +
                                   3 * (size_t)kHeads * kStaticMaxRows * kHeadDim * 2 +
                                   (size_t)kStaticMaxRows * kOutK * 2 + (size_t)kStaticMaxRows * kPairs * sizeof(float2) +
-                                  2 * (size_t)kStaticMaxRows * sizeof(float);
+                                  2 * (size_t)kStaticMaxRows * sizeof(float) +
+                                  2 * (size_t)kStaticMaxRows * (kDim / 16 + kOutK / 16);
 
 static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 

@@ -1,0 +1,249 @@
+"""GPU parity of the NVFP4 path (e2m1 values, e4m3 block scales per 16
+values, fp32 second-level scales) against the oracle (oracle/nvfp4.py).
+
+* The quantiser is integer work decided in fp32 by the same correctly
+  rounded operations on both sides: codes, block scales and second-level
+  scales bit-exact, in the layouts include/klein.h documents (codes two per
+  byte, block scales in 512-byte atoms).
+* The block-scaled GEMM core on the oracle's own quantisation of the same
+  inputs: only fp32 accumulation differs, <= 1e-4 * RMS.
+* The fused modLN + quantisation: fp32 rows on the GPU against the oracle's
+  fp64 rows, so a value within rounding of a code or scale boundary may take
+  the neighbouring one, rarely.
+* The NVFP4 block and a short denoise against the oracle's NVFP4 block:
+  bounds derived from the oracle's own sensitivity to the bf16 storage of the
+  out-projection input (tests/test_oracle_nvfp4.py, NVFP4_STORAGE_*).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import klein_inputs as ki  # noqa: E402
+import oracle as o  # noqa: E402
+from oracle import fp8, nvfp4  # noqa: E402
+from gpu_util import cosine, host, max_err_ratio, rms, to_bf16, to_f32, upload_block, upload_model, workspace  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from conftest import ensure_built
+    ensure_built()
+    import latent_flow_matching_joint_b200 as kb
+    return kb
+
+
+def unpack_codes(packed):
+    """uint8 [rows, cols/2] (value 2i in the low nibble) -> uint8 [rows, cols]."""
+    p = np.asarray(packed)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def unpack_scales(atoms, rows, cols):
+    """Block-scale atoms -> uint8 [rows, cols/16] (the layout of include/klein.h)."""
+    a = np.asarray(atoms)
+    r = np.arange(rows)[:, None]
+    b = np.arange(cols // 16)[None, :]
+    off = ((r // 128) * (cols // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+    return a[off]
+
+
+def _bf16_rows(seed, rows, cols):
+    rng = np.random.default_rng(seed)
+    mag = np.exp(rng.uniform(-10, 6, (rows, 1)))
+    a = (rng.standard_normal((rows, cols)) * mag).astype(np.float32)
+    a[:, 16:32] *= np.float32(2.0 ** -20)        # a block far below its row's range (subnormal block scale)
+    a[3] = 0.0                                   # an all-zero row
+    a[5, : cols // 2] = 0.0
+    a[9, 1] = np.float32(1e-30)
+    return ki.round_to_bf16(a)
+
+
+@pytest.mark.parametrize("rows,cols,mode", [(300, 3072, "matrix"), (130, 12288, "rows"), (17, 64, "rows"),
+                                            (40, 640, "matrix")])
+def test_quantiser_bit_exact(kb, rows, cols, mode):
+    a = _bf16_rows(rows + cols, rows, cols)
+    m = kb.NVFP4_ROWS if mode == "rows" else kb.NVFP4_MATRIX
+    codes, sf, g = kb.klein_quantize_nvfp4(to_bf16(a), m)
+    torch.cuda.synchronize()
+    c_ref, s_ref, g_ref = nvfp4.quantize(a, per_row=(mode == "rows"))
+    np.testing.assert_array_equal(unpack_codes(codes.cpu().numpy()), c_ref)
+    np.testing.assert_array_equal(unpack_scales(sf.cpu().numpy(), rows, cols), s_ref)
+    gg = g.cpu().numpy()
+    if mode == "rows":
+        np.testing.assert_array_equal(gg.view(np.uint32), np.asarray(g_ref, np.float32).ravel().view(np.uint32))
+        pad = (rows + 255) // 256 * 256
+    else:
+        assert gg[0] == np.float32(g_ref)
+        pad = (rows + 127) // 128 * 128
+    if pad > rows:   # padding rows of the last atom row hold scale 0
+        full = np.asarray(sf.cpu().numpy())
+        assert not unpack_scales(full, pad, cols)[rows:].any()
+
+
+def test_in_projection_order(kb):
+    # a block's w_in in the NVFP4 in-projection order: q, k, v rows as they
+    # are, then per 64-unit SwiGLU chunk its gate rows and its up rows
+    w = ki.block_weights(0, "joint.0")["w_in"]
+    codes, sf, g = kb.klein_quantize_nvfp4(to_bf16(w), kb.NVFP4_IN_PROJ)
+    torch.cuda.synchronize()
+    c_ref, s_ref, g_ref = nvfp4.quantize(w)
+    assert g.cpu().numpy()[0] == np.float32(g_ref)
+    got_c = codes.cpu().numpy()
+    got_s = sf.cpu().numpy()
+    d, f = 3 * ki.DIM, ki.MLP_HIDDEN
+    out_rows = np.array([0, 9215, 9216, 9216 + 63, 9216 + 64, 9216 + 127, 9216 + 128, 27647])
+    src_rows = np.array([0, 9215, d, d + 63, d + f, d + f + 63, d + 64, d + f + 9215])
+    np.testing.assert_array_equal(unpack_codes(got_c[out_rows]), c_ref[src_rows])
+    np.testing.assert_array_equal(unpack_scales(got_s, 27648, 3072)[out_rows], s_ref[src_rows])
+
+
+def test_quantiser_argument_errors(kb):
+    a = torch.zeros((4, 48), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kb.KleinError):          # cols not a multiple of 64
+        kb.klein_quantize_nvfp4(a, kb.NVFP4_MATRIX)
+    b = torch.zeros((27648, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kb.KleinError):          # the in-projection order needs [27648][3072]
+        kb.klein_quantize_nvfp4(b, kb.NVFP4_IN_PROJ)
+
+
+@pytest.mark.parametrize("m,n,k", [(300, 384, 512), (256, 128, 256), (1, 256, 3072), (513, 128, 768)])
+def test_gemm_nvfp4_core(kb, m, n, k):
+    rng = np.random.default_rng(m * 7 + n + k)
+    a = ki.round_to_bf16((rng.standard_normal((m, k)) * np.exp(rng.uniform(-2, 2, (m, 1)))).astype(np.float32))
+    b = ki.round_to_bf16((rng.standard_normal((n, k)) * 0.05).astype(np.float32))
+    qa = kb.klein_quantize_nvfp4(to_bf16(a), kb.NVFP4_ROWS)
+    qb = kb.klein_quantize_nvfp4(to_bf16(b), kb.NVFP4_MATRIX)
+    c = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
+    kb.klein_op_gemm_nvfp4(qa[0], qa[1], qa[2], qb[0], qb[1], qb[2], c)
+    torch.cuda.synchronize()
+    ref = nvfp4.fake_quant_rows(a) @ nvfp4.fake_quant(b).T
+    got = host(c)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - ref)) <= 1e-4 * rms(ref), np.max(np.abs(got - ref)) / rms(ref)
+
+
+def test_modln_nvfp4_codes(kb):
+    n_txt, n_img, n_ref = 100, 150, 30
+    n_total = n_txt + n_img + n_ref
+    rows = n_total - 10
+    x = ki.tokens(1, "nvfp4.modln", 2, n_total) * 3.0 + 0.5
+    mod = ki.modulation_vectors(1, "nvfp4.modln")
+    pad = (rows + 255) // 256 * 256
+    codes = torch.empty((2, rows, ki.DIM // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.full((2, pad * ki.DIM // 16), 0xAB, dtype=torch.uint8, device="cuda")
+    g = torch.empty((2, rows), dtype=torch.float32, device="cuda")
+    kb.klein_op_modln_nvfp4(to_f32(x), 10, rows, n_txt, n_img, to_f32(mod), codes, sf, g)
+    torch.cuda.synchronize()
+    modes = o.mode_of_rows(n_txt, n_img, n_ref)
+    h = o.modln(x, modes, mod.astype(np.float64))[:, 10:]
+    c_ref, s_ref, g_ref = nvfp4.quantize(h, per_row=True)
+    g_got = g.cpu().numpy()
+    assert np.max(np.abs(g_got / g_ref[..., 0] - 1)) <= 2e-6
+    sfh = sf.cpu().numpy()
+    s_got = np.stack([unpack_scales(sfh[b], pad, ki.DIM) for b in range(2)])
+    assert not s_got[:, rows:].any()             # padding rows of the last 256-row tile: scale 0
+    s_diff = s_got[:, :rows] != s_ref
+    assert s_diff.mean() <= 1e-3, s_diff.mean()
+    assert np.all(np.abs(s_got[:, :rows][s_diff].astype(int) - s_ref[s_diff].astype(int)) <= 1)
+    c_got = unpack_codes(codes.cpu().numpy())
+    # where the block scales agree, a differing code is the neighbouring one
+    same_blocks = np.repeat(~s_diff, 16, axis=-1)
+    diff = (c_got != c_ref) & same_blocks
+    assert diff.mean() <= 2e-3, diff.mean()
+    g_, r_ = c_got[diff].astype(int), c_ref[diff].astype(int)
+    at_zero = ((g_ & 7) == 0) | ((r_ & 7) == 0)
+    assert np.all(((g_ & 8) == (r_ & 8)) | at_zero)
+    assert np.all(np.abs((g_ & 7) - (r_ & 7)) <= 1)
+
+
+@pytest.fixture(scope="module")
+def nv_weights(kb):
+    w = ki.block_weights(0, "joint.0")
+    wd = kb.quantize_block_nvfp4(upload_block(w))
+    return nvfp4.quantize_block_weights(w), w, wd
+
+
+# Bounds of the NVFP4 block against the NVFP4 oracle: the GPU keeps the
+# [attention | SwiGLU] rows in bf16 before quantising them; on the oracle's
+# own block that moves the update by NVFP4_STORAGE_REL_MAX (0.04) of its RMS
+# and the worst element by NVFP4_STORAGE_WORST_MAX (0.2) x RMS(output)
+# (pinned in tests/test_oracle_nvfp4.py). Bounds: about 1.5x those.
+NV_REL = 0.06
+NV_MAX_ERR = 0.3
+
+NV_CASES = {
+    "config1": dict(batch=1, n_txt=80, img=(8, 8), refs=(), view="joint"),
+    "ragged_ref_b2": dict(batch=2, n_txt=77, img=(9, 7), refs=((3, 5),), view="joint"),
+    "stage1_image": dict(batch=1, n_txt=80, img=(12, 11), refs=(), view="img"),
+    "long_1024": dict(batch=1, n_txt=512, img=(32, 32), refs=(), view="joint"),
+}
+
+
+@pytest.mark.parametrize("name", list(NV_CASES))
+def test_nvfp4_block_matches_oracle(kb, nv_weights, name):
+    c = NV_CASES[name]
+    wq, w, wd = nv_weights
+    n_txt, (gh, gw), refs = c["n_txt"], c["img"], c["refs"]
+    n_img = gh * gw
+    n_ref = sum(h * ww for h, ww in refs)
+    n_total = n_txt + n_img + n_ref
+    seq = kb.make_seq(c["batch"], n_txt, gh, gw, refs)
+    x = ki.tokens(1, f"nvblock.{name}", c["batch"], n_total)
+    mod = ki.modulation_vectors(1, f"nvblock.{name}")
+    row0, rows = {"joint": (0, n_total), "img": (n_txt, n_img)}[c["view"]]
+    xd = to_f32(x)
+    pos = torch.empty((n_total, 4), dtype=torch.float32, device="cuda")
+    kb.klein_positions(seq, pos)
+    ws = workspace(kb.klein_block_workspace_size(c["batch"], rows))
+    kb.klein_block_forward(wd, xd, n_txt, n_img, pos, to_f32(mod), ws, row0=row0, rows=rows)
+    torch.cuda.synchronize()
+    got = host(xd)
+    posn = o.positions(n_txt, (gh, gw), refs)
+    modes = o.mode_of_rows(n_txt, n_img, n_ref)
+    sl = slice(row0, row0 + rows)
+    ref = o.block(x[:, sl], posn[sl], modes[sl], mod.astype(np.float64), wq)
+    g = got[:, sl]
+    assert np.all(np.isfinite(g))
+    d_got, d_ref = g - x[:, sl], ref - x[:, sl]
+    rel = rms(d_got - d_ref) / rms(d_ref)
+    assert rel <= NV_REL, rel
+    assert cosine(d_got, d_ref) >= 0.998
+    assert max_err_ratio(g, ref) <= NV_MAX_ERR, max_err_ratio(g, ref)
+    if name == "config1":
+        # the GPU computes the NVFP4 method, not another precision's: its
+        # distance to the NVFP4 oracle is well below that oracle's distance
+        # to the exact block (about 0.2 of the update)
+        exact = o.block(x[:, sl], posn[sl], modes[sl], mod.astype(np.float64), w)
+        assert rms(d_got - d_ref) < 0.5 * rms(exact - ref)
+
+
+def test_nvfp4_denoise_matches_oracle(kb):
+    m = ki.ModelWeights(seed=5, distilled=True, n_stage1=1, n_joint=2)
+    t = upload_model(m)
+    t["joint"] = [kb.quantize_block_nvfp4(b) for b in t["joint"]]
+    t["stage1"] = {k: [kb.quantize_block_nvfp4(b) for b in v] for k, v in t["stage1"].items()}
+    model = kb.KleinModel(t)
+    refs = ((4, 4),)
+    seq = kb.make_seq(1, 40, 6, 6, refs)
+    n_img, n_ref, n_total = kb.klein_seq_tokens(seq)
+    lat = ki.noise_latents(2, n_img)
+    text = ki.text_embeddings(1, 1, 40)
+    rl = ki.ref_latents(1, n_ref)
+    x = to_f32(lat)
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 1.0, seq, ws)
+    torch.cuda.synchronize()
+    ref = o.denoise(fp8.QuantizedModel(m, nvfp4.quantize_block_weights), lat, text, rl,
+                    o.positions(40, (6, 6), refs), 3)
+    got = host(x)
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert rms(got - ref) / rms(ref) <= NV_REL, rms(got - ref) / rms(ref)
+    assert max_err_ratio(got, ref) <= NV_MAX_ERR, max_err_ratio(got, ref)

@@ -151,7 +151,7 @@ def attention_bound(q, k, v, ref):
     return 2.0 ** -8 * (np.abs(ref) + o.attention(q, k, np.abs(v))) + 1e-6
 
 
-@pytest.mark.parametrize("batch,rows", [(1, 144), (2, 300), (1, 1), (1, 128), (1, 129)])
+@pytest.mark.parametrize("batch,rows", [(1, 144), (2, 300), (1, 1), (1, 128), (1, 129), (1, 513), (2, 700)])
 def test_attention_matches_oracle(kb, batch, rows):
     q, k, v, qd, kd, vtd = _attn_inputs(batch, rows, 24, f"{batch}.{rows}")
     out = torch.full((batch, rows, ki.DIM + ki.MLP_HIDDEN), float("nan"), dtype=torch.bfloat16, device="cuda")

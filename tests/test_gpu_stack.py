@@ -1,6 +1,6 @@
 """GPU parity of the modulation, the two-stage stack and the Euler sampler
 against the oracle, on random-init stacks of reduced depth (the full 5 + 28
-stack is exercised by the benchmark and by the slow test at the end)."""
+stack is compared with stored oracle outputs in test_gpu_full_size.py)."""
 import numpy as np
 import pytest
 
@@ -142,33 +142,6 @@ def test_denoise_argument_errors(kb, base):
     assert e.value.name == "KLEIN_ERR_INVALID_ARG"
 
 
-def test_full_depth_denoise_matches_stored_oracle(kb):
-    """The full 5 + 28 block distilled stack, 16 Euler steps, 80 text + 8x8
-    image tokens: final latents against the oracle's, stored by
-    tests/golden/make_denoise_golden.py (cosine >= 0.999)."""
-    import json
-    import os
-    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
-    path = os.path.join(here, "denoise_full_depth_80_8x8_16.npy")
-    meta = json.load(open(path.replace(".npy", ".json")))
-    m = ki.ModelWeights(seed=meta["weight_seed"], distilled=True)
-    t = upload_model(m, with_ref=False)
-    m._blocks.clear()
-    model = kb.KleinModel(t)
-    n_txt, (gh, gw) = meta["n_txt"], meta["grid"]
-    seq = kb.make_seq(1, n_txt, gh, gw)
-    x = to_f32(ki.noise_latents(meta["noise_seed"], gh * gw))
-    text = to_bf16(ki.text_embeddings(meta["text_seed"], 1, n_txt))
-    ws = workspace(kb.klein_stack_workspace_size(seq))
-    kb.klein_denoise(model, x, text, None, meta["steps"], 1.0, seq, ws)
-    torch.cuda.synchronize()
-    ref = np.load(path)
-    got = host(x)
-    assert np.all(np.isfinite(got))
-    assert cosine(got, ref) >= 0.999, cosine(got, ref)
-    assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)
-
-
 def test_stack_forward_with_text_projection(kb):
     # text given as the stacked encoder hidden states (8 x 2560 per token),
     # projected to 3072 by the model's txt_in; batch 2 (distinct texts)
@@ -207,3 +180,67 @@ def test_denoise_base_with_reference_uses_stage1_cache(kb):
     ref = o.denoise(m, lat, text, rl, o.positions(20, (5, 4), refs), 3, cfg=2.0)
     assert cosine(host(x), ref) >= 0.999
     assert max_err_ratio(host(x), ref) <= 5e-2
+
+
+@pytest.fixture(scope="module")
+def distilled_refs(kb):
+    m = ki.ModelWeights(seed=5, distilled=True, n_stage1=1, n_joint=2)
+    t = upload_model(m)
+    return m, t, kb.KleinModel(t)
+
+
+THREE_REFS = ((4, 6), (3, 5), (6, 2))   # three reference images, each its own grid size
+
+
+def test_stack_forward_three_references(kb, distilled_refs):
+    # an edit with three references of different sizes: each takes its own l
+    # offset (-1, -2, -3) and all join the reference stream of stage 1
+    m, _, model = distilled_refs
+    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 1, 48, 5, 7, THREE_REFS, "refs3")
+    assert n_ref == 24 + 15 + 12
+    v = torch.full((1, n_img, 128), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_stack_forward(model, to_f32(lat), to_bf16(text), to_f32(rl), 0.8, 0.6, seq, v, ws)
+    torch.cuda.synchronize()
+    ref = o.transformer(m, lat, text, rl, o.positions(48, (5, 7), THREE_REFS), 0.8, 0.6)
+    got = host(v)
+    assert np.all(np.isfinite(got))
+    assert cosine(got, ref) >= 0.999, cosine(got, ref)
+    assert max_err_ratio(got, ref) <= 5e-2, max_err_ratio(got, ref)
+
+
+def test_denoise_three_references(kb, distilled_refs):
+    m, _, model = distilled_refs
+    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 1, 32, 4, 6, THREE_REFS, "refs3den")
+    x = to_f32(lat)
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, to_bf16(text), to_f32(rl), 3, 1.0, seq, ws)
+    torch.cuda.synchronize()
+    ref = o.denoise(m, lat, text, rl, o.positions(32, (4, 6), THREE_REFS), 3)
+    assert cosine(host(x), ref) >= 0.999
+    assert max_err_ratio(host(x), ref) <= 5e-2
+
+
+def test_denoise_x0_preview_every_step(kb, distilled):
+    # the x0 preview x - sigma v of every step (before its update), as the
+    # pages' preview block shows after each denoiser call
+    m, _, model = distilled
+    seq, n_img, n_ref, n_total, lat, text, rl = _seq_inputs(kb, 1, 40, 6, 6, (), "x0steps")
+    steps = 3
+    x = to_f32(lat)
+    x0 = torch.full((steps, n_img, 128), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(kb.klein_stack_workspace_size(seq))
+    kb.klein_denoise(model, x, to_bf16(text), None, steps, 1.0, seq, ws, x0_out=x0, x0_every_step=True)
+    torch.cuda.synchronize()
+    previews = {}
+
+    def on_step(i, xi, vi, s):
+        previews[i] = o.x0_preview(xi, vi, s)
+
+    ref = o.denoise(m, lat, text, None, o.positions(40, (6, 6)), steps, on_step=on_step)
+    assert cosine(host(x), ref) >= 0.999
+    got = host(x0)
+    for i in range(steps):
+        assert np.all(np.isfinite(got[i])), i
+        assert cosine(got[i], previews[i]) >= 0.999, (i, cosine(got[i], previews[i]))
+        assert max_err_ratio(got[i], previews[i]) <= 5e-2, (i, max_err_ratio(got[i], previews[i]))

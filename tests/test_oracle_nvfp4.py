@@ -148,3 +148,43 @@ def test_nvfp4_block_tracks_exact_block():
     # row-subset evaluation still equals the full block (per-row activation scales)
     rows = np.array([0, 5, 79, 80, 143])
     np.testing.assert_allclose(o.block(x, pos, modes, mod, wq, rows=rows), quant[:, rows], rtol=0, atol=1e-12)
+
+
+# Effect, on the oracle's own NVFP4 block, of one bf16 rounding of the
+# concatenated [attention | SwiGLU] rows ahead of their NVFP4 quantisation
+# (what the GPU does: it stores those rows in bf16 before quantising them),
+# relative to the block update (RMS) and to RMS(output) at the worst element.
+# The GPU tests derive their NVFP4 bounds from these (about 2x and 1.5x).
+NVFP4_STORAGE_REL_MAX = 0.04
+NVFP4_STORAGE_WORST_MAX = 0.2
+
+
+def test_nvfp4_block_sensitivity_to_bf16_storage_of_the_out_projection_input():
+    import klein_inputs as ki
+    import oracle as o
+    from oracle.klein import DIM, HEAD_DIM, HEADS, _split_w_in, attention, modln, rms_norm, rope, swiglu
+    w = ki.block_weights(0, "joint.0")
+    wq = nvfp4.quantize_block_weights(w)
+    x = ki.tokens(1, "nvfp4block.config1", 1, 144)
+    mod = ki.modulation_vectors(1, "nvfp4block.config1").astype(np.float64)
+    pos = o.positions(80, (8, 8))
+    modes = o.mode_of_rows(80, 64, 0)
+    ref = o.block(x, pos, modes, mod, wq)
+    # the same block recomposed from the oracle's steps, then with the
+    # concatenated rows rounded to bf16 before their quantisation
+    h = nvfp4.fake_quant_rows(modln(x, modes, mod))
+    w_q, w_k, w_v, w_g, w_u = _split_w_in(nvfp4.dequantize(*wq["w_in_nv"]))
+    q = rope(rms_norm((h @ w_q.T).reshape(1, 144, HEADS, HEAD_DIM), w["q_norm"]), pos)
+    k = rope(rms_norm((h @ w_k.T).reshape(1, 144, HEADS, HEAD_DIM), w["k_norm"]), pos)
+    v = (h @ w_v.T).reshape(1, 144, HEADS, HEAD_DIM)
+    a_cat = np.concatenate([attention(q, k, v).reshape(1, 144, DIM), swiglu(h @ w_g.T, h @ w_u.T)], -1)
+    w_out = nvfp4.dequantize(*wq["w_out_nv"])
+    same = x + mod[modes, 2] * (nvfp4.fake_quant_rows(a_cat) @ w_out.T)
+    assert np.max(np.abs(same - ref)) <= 1e-9 * np.sqrt(np.mean(ref ** 2))   # the recomposition is the block
+    a_bf = ki.round_to_bf16(a_cat.astype(np.float32)).astype(np.float64)
+    pert = x + mod[modes, 2] * (nvfp4.fake_quant_rows(a_bf) @ w_out.T)
+    r = lambda a: float(np.sqrt(np.mean(a * a)))  # noqa: E731
+    rel = r(pert - ref) / r(ref - x)
+    worst = float(np.max(np.abs(pert - ref))) / r(ref)
+    assert 0.005 < rel <= NVFP4_STORAGE_REL_MAX, rel
+    assert 0.02 < worst <= NVFP4_STORAGE_WORST_MAX, worst
