@@ -89,9 +89,10 @@ __device__ __forceinline__ void e4m3_row_scales(float amax, float& inv, float& s
 
 // modLN with the output quantised: one warp per row, as modln_kernel. The
 // modulated row stays in registers between the row maximum and the codes
-// (one block of 8 warps per SM: 8 x 32 lanes x 24 x 16 bytes of loads in
-// flight per SM still cover the HBM latency).
-__global__ void __launch_bounds__(256, 1) modln_e4m3_kernel(const float* __restrict__ x, long long x_bstride,
+// (two blocks of 8 warps per SM; at 128 registers ptxas spills 28 bytes of
+// the row, and the kernel is still faster than at one block per SM because
+// twice the loads are in flight).
+__global__ void __launch_bounds__(256, 2) modln_e4m3_kernel(const float* __restrict__ x, long long x_bstride,
                                                          int x_row0, uint32_t* __restrict__ codes,
                                                          float* __restrict__ scale, int batch, int rows,
                                                          int n_txt, int n_img, const float* __restrict__ mod,
