@@ -44,8 +44,13 @@ constexpr int kStage = kStageA + kStageB + 2 * kStageSF;
 constexpr int kStages = 7;
 constexpr int kTileBytes = kStages * kStage;
 constexpr int kSmem = kTileBytes + 1024 + 256;
-constexpr uint32_t kTmemCols = 512;  // accumulators 2 x 128, A scales 16, B scales 16 columns
-constexpr uint32_t kSfaCol = 256, kSfbCol = 272;
+// accumulators 2 x 128 columns, then one 32-column scale slot per smem stage
+// (A scales 16 columns, B scales 16): a stage's scale copy must not write
+// columns that MMAs still in the tensor pipe read, or every stage would wait
+// for the pipe to drain
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCol0 = 256, kSfSlot = 32;
+static_assert(kSfCol0 + kStages * kSfSlot <= kTmemCols, "scale slots exceed the TMEM allocation");
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr float kG = 448.0f * 6.0f;
@@ -614,17 +619,20 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
           const uint32_t b0 = a0 + nv::kStageA;
           const uint32_t sfa0 = b0 + nv::kStageB;
           const uint32_t sfb0 = sfa0 + nv::kStageSF;
-          // this stage's scales into tensor memory (in order with the MMAs
-          // that read them, after the previous stage's MMAs)
+          // this stage's scales into the stage's own tensor-memory slot (the
+          // copies run in order with the MMAs; the slot was last read by the
+          // MMAs of the stage kStages back, long finished)
+          const uint32_t sfa_t = tmem_base + nv::kSfCol0 + nv::kSfSlot * stage;
+          const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            tmem_cp_atom_pair(tmem_base + nv::kSfaCol + 4 * k, sf_atom_desc(sfa0 + 512 * k));
-            tmem_cp_atom_pair(tmem_base + nv::kSfbCol + 4 * k, sf_atom_desc(sfb0 + 512 * k));
+            tmem_cp_atom_pair(sfa_t + 4 * k, sf_atom_desc(sfa0 + 512 * k));
+            tmem_cp_atom_pair(sfb_t + 4 * k, sf_atom_desc(sfb0 + 512 * k));
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_nvfp4_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, tmem_base + nv::kSfaCol + 4 * k,
-                            tmem_base + nv::kSfbCol + 4 * k, (kb | k) != 0);
+            umma_nvfp4_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, sfa_t + 4 * k, sfb_t + 4 * k,
+                            (kb | k) != 0);
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == nv::kStages) { stage = 0; phase ^= 1; }
         }
