@@ -27,10 +27,14 @@
 // M = 256 from the two CTAs' 128 A rows, N = 128 from 64 B rows of each CTA;
 // K in stages of 256 values (128 bytes per row, one 128-byte swizzle row);
 // per stage each CTA also loads its A rows' scales (4 atoms) and the tile's
-// B scales (4 atoms, the same in both CTAs), which the MMA thread copies to
-// tensor memory ahead of the stage's four K = 64 MMAs
-// (tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16). Two
-// 128-column accumulators let the epilogue of one tile overlap the next.
+// B scales (4 atoms, the same in both CTAs). A scale warp copies them to the
+// stage's slot in tensor memory and signals the MMA thread, which then
+// issues the stage's four K = 64 MMAs
+// (tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16). The copies
+// run from their own thread because, queued by the MMA thread in front of
+// the MMAs, they took about as long as the MMAs themselves. Eight stages of
+// 28 KB per CTA; two 128-column accumulators let the epilogue of one tile
+// overlap the next.
 #include "common.cuh"
 #include "internal.h"
 
@@ -41,18 +45,20 @@ constexpr int kStageA = 128 * 128;   // this CTA's 128 A rows x 128 bytes
 constexpr int kStageB = 64 * 128;    // this CTA's 64 B rows x 128 bytes
 constexpr int kStageSF = 4 * 512;    // four scale atoms (K = 256 values)
 constexpr int kStage = kStageA + kStageB + 2 * kStageSF;
-constexpr int kStages = 7;
+constexpr int kStages = 8;
 constexpr int kTileBytes = kStages * kStage;
 constexpr int kSmem = kTileBytes + 1024 + 256;
 // accumulators 2 x 128 columns, then one 32-column scale slot per smem stage
-// (A scales 16 columns, B scales 16): a stage's scale copy must not write
-// columns that MMAs still in the tensor pipe read, or every stage would wait
-// for the pipe to drain
+// (A scales 16 columns, B scales 16). The scale copies come from a thread
+// of their own, so nothing orders them after the MMAs of earlier stages:
+// giving every stage its own slot is what keeps a copy from overwriting
+// scales an MMA still reads.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256, kSfSlot = 32;
 static_assert(kSfCol0 + kStages * kSfSlot <= kTmemCols, "scale slots exceed the TMEM allocation");
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kSfWarp = 2 + kEpiWarps;  // copies the block scales to tensor memory
+constexpr int kThreads = 32 * (kSfWarp + 1);
 constexpr float kG = 448.0f * 6.0f;
 }  // namespace nv
 
@@ -524,7 +530,10 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
   uint64_t* acc_full = empty + nv::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = drain + 1;  // [kStages]: the stage's scales are in tensor memory
+  uint64_t* sf_drain = sf_ready + nv::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_drain + 1);
+  static_assert((2 * nv::kStages + 5 + nv::kStages + 1) * 8 + 4 <= 256, "barriers exceed their shared-memory area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -541,6 +550,8 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
       mbar_init(&acc_empty[a], 2 * 32 * nv::kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < nv::kStages; ++s) mbar_init(&sf_ready[s], 1);
+    mbar_init(sf_drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
@@ -613,22 +624,17 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
         const uint32_t d = tmem_base + acc * 128;
         bool ok = true;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, 0x133)) { ok = false; break; }
+          // operands in shared memory, and their scales in the stage's
+          // tensor-memory slot (copied by the scale warp)
+          if (!mbar_wait(&full[stage], phase, 0x133) || !mbar_wait(&sf_ready[stage], phase, 0x137)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * nv::kStage);
           const uint32_t b0 = a0 + nv::kStageA;
-          const uint32_t sfa0 = b0 + nv::kStageB;
-          const uint32_t sfb0 = sfa0 + nv::kStageSF;
-          // this stage's scales into the stage's own tensor-memory slot (the
-          // copies run in order with the MMAs; the slot was last read by the
-          // MMAs of the stage kStages back, long finished)
           const uint32_t sfa_t = tmem_base + nv::kSfCol0 + nv::kSfSlot * stage;
           const uint32_t sfb_t = sfa_t + 16;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            tmem_cp_atom_pair(sfa_t + 4 * k, sf_atom_desc(sfa0 + 512 * k));
-            tmem_cp_atom_pair(sfb_t + 4 * k, sf_atom_desc(sfb0 + 512 * k));
-          }
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_nvfp4_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, sfa_t + 4 * k, sfb_t + 4 * k,
@@ -641,6 +647,35 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
       }
       umma_commit_pair(drain, 0x1);
       mbar_wait(drain, 0, 0x136);
+    }
+  } else if (warp == nv::kSfWarp) {
+    // Block scales to tensor memory, from a thread of their own: issued by
+    // the MMA thread, each stage's eight copies sat in its tensor-core queue
+    // ahead of the MMAs and cost about as much time as the MMAs. The copy
+    // for stage s of step n lands in slot s, which the MMAs of step
+    // n - kStages last read; those completed before the producer could
+    // refill stage s, which this thread waited for.
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const int steps = ((total - pair + npairs - 1) / npairs) * g.k_blocks;
+      for (int n = 0; n < steps; ++n) {
+        if (!mbar_wait(&full[stage], phase, 0x138)) break;
+        tc_fence_after();
+        const uint32_t sfa0 = smem_u32(smem + stage * nv::kStage) + nv::kStageA + nv::kStageB;
+        const uint32_t sfb0 = sfa0 + nv::kStageSF;
+        const uint32_t sfa_t = tmem_base + nv::kSfCol0 + nv::kSfSlot * stage;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          tmem_cp_atom_pair(sfa_t + 4 * k, sf_atom_desc(sfa0 + 512 * k));
+          tmem_cp_atom_pair(sfa_t + 16 + 4 * k, sf_atom_desc(sfb0 + 512 * k));
+        }
+        umma_commit_pair(&sf_ready[stage], 0x1);
+        if (++stage == nv::kStages) { stage = 0; phase ^= 1; }
+      }
+      // every copy issued here has completed before tensor memory is freed
+      umma_commit_pair(sf_drain, 0x1);
+      mbar_wait(sf_drain, 0, 0x139);
     }
   } else {
     const int quarter = warp & 3;

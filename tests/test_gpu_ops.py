@@ -166,6 +166,36 @@ def test_attention_matches_oracle(kb, batch, rows):
     assert torch.isnan(out[:, :, ki.DIM:]).all()
 
 
+@pytest.mark.parametrize("batch,rows", [(1, 200), (2, 700)])
+def test_attention_rescales_mid_tile(kb, batch, rows):
+    """Scores that climb along the keys: q . k_j grows by about 2 per key, so
+    a row's maximum (in exp2 units) rises by ~16 every 64 keys, far past
+    the kernel's lazy-rescale threshold of 8, and the running maximum moves
+    (and O is rescaled) in every key tile, the last one included. The
+    per-row factor s_i in [0, 1.5] leaves some rows of each warp below the
+    threshold, so rows that rescale and rows that do not share a warp."""
+    rp = (rows + 127) // 128 * 128
+    s_i = np.linspace(0.0, 1.5, rows)[None, :, None, None]
+    ramp = (np.arange(rows) / 64.0)[None, :, None, None]
+    q = ki.round_to_bf16(s_i * (1.0 + 0.1 * ki.normal(8, f"attn.rq.{rows}", (batch, rows, 24, 128))))
+    k = ki.round_to_bf16(ramp * (1.0 + 0.1 * ki.normal(8, f"attn.rk.{rows}", (batch, rows, 24, 128))))
+    v = ki.normal(8, f"attn.rv.{rows}", (batch, rows, 24, 128))
+    qd = torch.zeros((batch, 24, rp, 128), dtype=torch.bfloat16, device="cuda")
+    kd = torch.zeros_like(qd)
+    vtd = torch.zeros((batch, 24, 128, rp), dtype=torch.bfloat16, device="cuda")
+    qd[:, :, :rows] = to_bf16(q).permute(0, 2, 1, 3)
+    kd[:, :, :rows] = to_bf16(k).permute(0, 2, 1, 3)
+    vtd[:, :, :, :rows] = to_bf16(v).permute(0, 2, 3, 1)
+    out = torch.empty((batch, rows, ki.DIM), dtype=torch.bfloat16, device="cuda")
+    kb.klein_op_attention(qd, kd, vtd, rows, out)
+    torch.cuda.synchronize()
+    got = host(out).reshape(batch, rows, 24, 128)
+    ref = o.attention(q, k, v)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - ref) <= attention_bound(q, k, v, ref))
+    assert cosine(got, ref) >= 0.9999
+
+
 def test_attention_long_sampled(kb):
     rows = 4608
     q, k, v, qd, kd, vtd = _attn_inputs(1, rows, 24, "long")
