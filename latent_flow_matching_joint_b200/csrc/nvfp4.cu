@@ -23,7 +23,8 @@
 //          column (r % 128) / 32, byte b. Rows past the matrix up to a
 //          multiple of 128 hold scale 0.
 //
-// The GEMM (gemm_nvfp4_kernel) runs on CTA pairs: 256 x 128 output tiles,
+// The GEMM (gemm_nvfp4_kernel) runs on CTA pairs: 256 x 128 output tiles
+// (256 x 256, two N = 128 halves per A stage, for the out-projection),
 // M = 256 from the two CTAs' 128 A rows, N = 128 from 64 B rows of each CTA;
 // K in stages of 256 values (128 bytes per row, one 128-byte swizzle row);
 // per stage each CTA also loads its A rows' scales (4 atoms) and the tile's
@@ -32,30 +33,45 @@
 // issues the stage's four K = 64 MMAs
 // (tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16). The copies
 // run from their own thread because, queued by the MMA thread in front of
-// the MMAs, they took about as long as the MMAs themselves. Eight stages of
-// 28 KB per CTA; two 128-column accumulators let the epilogue of one tile
-// overlap the next.
+// the MMAs, they took about as long as the MMAs themselves. Tile
+// configurations in nv::Cfg.
 #include "common.cuh"
 #include "internal.h"
 
 namespace klein {
 
 namespace nv {
-constexpr int kStageA = 128 * 128;   // this CTA's 128 A rows x 128 bytes
-constexpr int kStageB = 64 * 128;    // this CTA's 64 B rows x 128 bytes
-constexpr int kStageSF = 4 * 512;    // four scale atoms (K = 256 values)
-constexpr int kStage = kStageA + kStageB + 2 * kStageSF;
-constexpr int kStages = 8;
-constexpr int kTileBytes = kStages * kStage;
-constexpr int kSmem = kTileBytes + 1024 + 256;
-// accumulators 2 x 128 columns, then one 32-column scale slot per smem stage
-// (A scales 16 columns, B scales 16). The scale copies come from a thread
-// of their own, so nothing orders them after the MMAs of earlier stages:
-// giving every stage its own slot is what keeps a copy from overwriting
-// scales an MMA still reads.
+// Tile configurations. Narrow (in-projection, plain GEMM): 256 x 128 tiles,
+// two 128-column accumulators so that the epilogue of one tile overlaps the
+// next, eight stages. Wide (out-projection): 256 x 256 tiles as two N = 128
+// halves sharing each A stage, one 256-column accumulator, five stages; its
+// epilogue is light next to 48 K stages a tile, so serialising it costs
+// little, and each stage carries twice the MMA work per A byte.
+template <bool WIDE>
+struct Cfg {
+  static constexpr int kHalves = WIDE ? 2 : 1;          // N = 128 halves per tile
+  static constexpr int kStageA = 128 * 128;             // this CTA's 128 A rows x 128 bytes
+  static constexpr int kStageB = kHalves * 64 * 128;    // this CTA's 64 B rows of each half
+  static constexpr int kStageSFA = 4 * 512;             // four scale atoms (K = 256 values)
+  static constexpr int kStageSFB = kHalves * 4 * 512;   // the same for each half's 128 B rows
+  static constexpr int kStage = kStageA + kStageB + kStageSFA + kStageSFB;
+  static constexpr int kStages = WIDE ? 5 : 8;
+  static constexpr int kAccs = WIDE ? 1 : 2;
+  static constexpr int kTileBytes = kStages * kStage;
+  static constexpr int kSmem = kTileBytes + 1024 + 256;
+  // TMEM: accumulators in columns 0..255, then one scale slot per smem
+  // stage (A scales 16 columns, then 16 per half for B). The scale copies
+  // come from a thread of their own, so nothing orders them after the MMAs
+  // of earlier stages: giving every stage its own slot is what keeps a copy
+  // from overwriting scales an MMA still reads.
+  static constexpr uint32_t kSfCol0 = 256;
+  static constexpr uint32_t kSfSlot = 16 + 16 * kHalves;
+  static_assert(kAccs * 128 * kHalves == 256, "accumulators fill columns 0..255");
+  static_assert(kSfCol0 + kStages * kSfSlot <= 512, "scale slots exceed the TMEM allocation");
+  static_assert(kSmem <= 227 * 1024, "stages exceed shared memory");
+  static_assert((3 * kStages + 5 + 1) * 8 + 4 <= 256, "barriers exceed their shared-memory area");
+};
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfCol0 = 256, kSfSlot = 32;
-static_assert(kSfCol0 + kStages * kSfSlot <= kTmemCols, "scale slots exceed the TMEM allocation");
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarp = 2 + kEpiWarps;  // copies the block scales to tensor memory
 constexpr int kThreads = 32 * (kSfWarp + 1);
@@ -523,17 +539,17 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                       const GemmArgs g) {
+  using C = nv::Cfg<EPI == kEpiResid>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + nv::kTileBytes);
-  uint64_t* empty = full + nv::kStages;
-  uint64_t* acc_full = empty + nv::kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kTileBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* sf_ready = empty + C::kStages;  // [kStages]: the stage's scales are in tensor memory
+  uint64_t* acc_full = sf_ready + C::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* sf_ready = drain + 1;  // [kStages]: the stage's scales are in tensor memory
-  uint64_t* sf_drain = sf_ready + nv::kStages;
+  uint64_t* sf_drain = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_drain + 1);
-  static_assert((2 * nv::kStages + 5 + nv::kStages + 1) * 8 + 4 <= 256, "barriers exceed their shared-memory area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -541,16 +557,16 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
   const bool leader = rank == 0;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < nv::kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 2 * 32 * nv::kEpiWarps);
     }
     mbar_init(drain, 1);
-    for (int s = 0; s < nv::kStages; ++s) mbar_init(&sf_ready[s], 1);
     mbar_init(sf_drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&map_a);
@@ -569,8 +585,10 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
   pdl_trigger();
   pdl_wait();  // operands and outputs are touched only after the previous kernel completes
 
+  // g.n_tiles counts 128-column tiles; a wide tile covers kHalves of them
+  const int n_tiles = g.n_tiles / C::kHalves;
   const int m_tiles = g.batch * g.m_tiles_per_b;
-  const int total = m_tiles * g.n_tiles;
+  const int total = m_tiles * n_tiles;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
   constexpr uint32_t idesc = idesc_nvfp4(256, 128);
@@ -582,34 +600,38 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
       uint32_t phase = 0;
       StageLog log;
       for (int tile = pair; tile < total; tile += npairs) {
-        const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
-        const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
+        const int m_idx = g.n_fastest ? tile / n_tiles : tile % m_tiles;
+        const int n_idx = g.n_fastest ? tile % n_tiles : tile / m_tiles;
         const int b = m_idx / g.m_tiles_per_b;
         const int mt = m_idx % g.m_tiles_per_b;
         const int row0 = mt * 256 + 128 * static_cast<int>(rank);
-        const int brow = n_idx * 128 + 64 * static_cast<int>(rank);
         // scale atoms: this CTA's 128 A rows (atom row 2 mt + rank of batch
-        // item b), and the tile's 128 B rows (atom row n_idx)
+        // item b), and each half's 128 B rows (atom row of that half)
         const int sfa_row = (b * g.m_tiles_per_b * 2 + 2 * mt + static_cast<int>(rank)) * k_atoms;
-        const int sfb_row = n_idx * k_atoms;
         bool ok = true;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, 0x131)) { ok = false; break; }
           if (leader) {
-            mbar_arrive_expect_tx(&full[stage], 2 * nv::kStage);
+            mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
             log.armed(stage, phase);
           }
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-          uint8_t* sa = smem + stage * nv::kStage;
+          uint8_t* sa = smem + stage * C::kStage;
+          uint8_t* ssfa = sa + C::kStageA + C::kStageB;
           tma_load_3d_pair(sa, &map_a, bar, kb * 128, row0, b);
-          tma_load_2d_pair(sa + nv::kStageA, &map_b, bar, kb * 128, brow);
-          tma_load_2d_pair(sa + nv::kStageA + nv::kStageB, &map_sfa, bar, 0, sfa_row + 4 * kb);
-          tma_load_2d_pair(sa + nv::kStageA + nv::kStageB + nv::kStageSF, &map_sfb, bar, 0, sfb_row + 4 * kb);
-          if (++stage == nv::kStages) { stage = 0; phase ^= 1; }
+          tma_load_2d_pair(ssfa, &map_sfa, bar, 0, sfa_row + 4 * kb);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            const int n128 = n_idx * C::kHalves + h;
+            tma_load_2d_pair(sa + C::kStageA + h * 64 * 128, &map_b, bar, kb * 128,
+                             n128 * 128 + 64 * static_cast<int>(rank));
+            tma_load_2d_pair(ssfa + C::kStageSFA + h * 4 * 512, &map_sfb, bar, 0, n128 * k_atoms + 4 * kb);
+          }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
       }
-      if (leader) log.drain(full, nv::kStages, 0x135);
+      if (leader) log.drain(full, C::kStages, 0x135);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -617,8 +639,8 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       for (int tile = pair; tile < total; tile += npairs, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = C::kAccs == 2 ? (it & 1) : 0;
+        const uint32_t acc_phase = C::kAccs == 2 ? ((it >> 1) & 1) : (it & 1);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, 0x132)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * 128;
@@ -631,16 +653,18 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * nv::kStage);
-          const uint32_t b0 = a0 + nv::kStageA;
-          const uint32_t sfa_t = tmem_base + nv::kSfCol0 + nv::kSfSlot * stage;
-          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t a0 = smem_u32(smem + stage * C::kStage);
+          const uint32_t b0 = a0 + C::kStageA;
+          const uint32_t sfa_t = tmem_base + C::kSfCol0 + C::kSfSlot * stage;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_nvfp4_pair(d, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc, sfa_t + 4 * k, sfb_t + 4 * k,
-                            (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              umma_nvfp4_pair(d + 128 * h, sw128_desc(a0 + 32 * k), sw128_desc(b0 + h * 64 * 128 + 32 * k), idesc,
+                              sfa_t + 4 * k, sfa_t + 16 + 16 * h + 4 * k, (kb | k) != 0);
+          }
           umma_commit_pair(&empty[stage], 0x3);
-          if (++stage == nv::kStages) { stage = 0; phase ^= 1; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         umma_commit_pair(&acc_full[acc], 0x3);
@@ -650,11 +674,11 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
     }
   } else if (warp == nv::kSfWarp) {
     // Block scales to tensor memory, from a thread of their own: issued by
-    // the MMA thread, each stage's eight copies sat in its tensor-core queue
-    // ahead of the MMAs and cost about as much time as the MMAs. The copy
-    // for stage s of step n lands in slot s, which the MMAs of step
-    // n - kStages last read; those completed before the producer could
-    // refill stage s, which this thread waited for.
+    // the MMA thread, each stage's copies sat in its tensor-core queue ahead
+    // of the MMAs and cost about as much time as the MMAs. The copy for
+    // stage s of step n lands in slot s, which the MMAs of step n - kStages
+    // last read; those completed before the producer could refill stage s,
+    // which this thread waited for.
     if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
@@ -662,16 +686,17 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
       for (int n = 0; n < steps; ++n) {
         if (!mbar_wait(&full[stage], phase, 0x138)) break;
         tc_fence_after();
-        const uint32_t sfa0 = smem_u32(smem + stage * nv::kStage) + nv::kStageA + nv::kStageB;
-        const uint32_t sfb0 = sfa0 + nv::kStageSF;
-        const uint32_t sfa_t = tmem_base + nv::kSfCol0 + nv::kSfSlot * stage;
+        const uint32_t sfa0 = smem_u32(smem + stage * C::kStage) + C::kStageA + C::kStageB;
+        const uint32_t sfa_t = tmem_base + C::kSfCol0 + C::kSfSlot * stage;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           tmem_cp_atom_pair(sfa_t + 4 * k, sf_atom_desc(sfa0 + 512 * k));
-          tmem_cp_atom_pair(sfa_t + 16 + 4 * k, sf_atom_desc(sfb0 + 512 * k));
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h)
+            tmem_cp_atom_pair(sfa_t + 16 + 16 * h + 4 * k, sf_atom_desc(sfa0 + C::kStageSFA + h * 4 * 512 + 512 * k));
         }
         umma_commit_pair(&sf_ready[stage], 0x1);
-        if (++stage == nv::kStages) { stage = 0; phase ^= 1; }
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
       // every copy issued here has completed before tensor memory is freed
       umma_commit_pair(sf_drain, 0x1);
@@ -683,19 +708,23 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
     const int part = (warp - 2) / 4;
     int it = 0;
     for (int tile = pair; tile < total; tile += npairs, ++it) {
-      const int m_idx = g.n_fastest ? tile / g.n_tiles : tile % m_tiles;
-      const int n_idx = g.n_fastest ? tile % g.n_tiles : tile / m_tiles;
+      const int m_idx = g.n_fastest ? tile / n_tiles : tile % m_tiles;
+      const int n_idx = g.n_fastest ? tile % n_tiles : tile / m_tiles;
       const int b = m_idx / g.m_tiles_per_b;
       const int r = (m_idx % g.m_tiles_per_b) * 256 + 128 * static_cast<int>(rank) + rloc;
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = C::kAccs == 2 ? (it & 1) : 0;
+      const uint32_t acc_phase = C::kAccs == 2 ? ((it >> 1) & 1) : (it & 1);
       if (!mbar_wait(&acc_full[acc], acc_phase, 0x134)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * 128 + (static_cast<uint32_t>(quarter * 32) << 16);
       const float ga = r < g.rows ? __ldg(g.a_scale + (long long)b * g.rows + r) : 0.f;
-      if (EPI == kEpiF32) nv_epi_store(taddr, g, b, r, n_idx, part, ga);
-      else if (EPI == kEpiQKV) nv_epi_qkv(taddr, g, b, r, n_idx, part, ga);
-      else nv_epi_resid(taddr, g, b, r, n_idx, part, ga);
+#pragma unroll 1
+      for (int h = 0; h < C::kHalves; ++h) {
+        const int n128 = n_idx * C::kHalves + h;  // the 128-column tile this half covers
+        if (EPI == kEpiF32) nv_epi_store(taddr + 128 * h, g, b, r, n128, part, ga);
+        else if (EPI == kEpiQKV) nv_epi_qkv(taddr + 128 * h, g, b, r, n128, part, ga);
+        else nv_epi_resid(taddr + 128 * h, g, b, r, n128, part, ga);
+      }
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
     }
@@ -714,12 +743,14 @@ __global__ void __launch_bounds__(nv::kThreads, 1)
 template <int EPI>
 static int launch_nvfp4_one(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msfa,
                             const CUtensorMap& msfb, const GemmArgs& g, cudaStream_t s) {
+  using C = nv::Cfg<EPI == kEpiResid>;
+  if (g.n_tiles % C::kHalves != 0) return -2;  // a wide tile covers two 128-column tiles
   static int max_pairs_dev[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0) return -1;
   int& max_pairs = max_pairs_dev[dev];
   if (max_pairs == 0) {
-    if (cudaFuncSetAttribute(gemm_nvfp4_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, nv::kSmem) !=
+    if (cudaFuncSetAttribute(gemm_nvfp4_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
         cudaSuccess)
       return -1;
     cudaLaunchConfig_t cfg = {};
@@ -730,17 +761,17 @@ static int launch_nvfp4_one(const CUtensorMap& ma, const CUtensorMap& mb, const 
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * (num_sms() / 2));
     cfg.blockDim = dim3(nv::kThreads);
-    cfg.dynamicSmemBytes = nv::kSmem;
+    cfg.dynamicSmemBytes = C::kSmem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel<EPI>, &cfg) != cudaSuccess || n < 1) return -1;
     max_pairs = n;
   }
-  const int total = g.batch * g.m_tiles_per_b * g.n_tiles;
+  const int total = g.batch * g.m_tiles_per_b * (g.n_tiles / C::kHalves);
   if (total <= 0) return 0;
   const int pairs = total < max_pairs ? total : max_pairs;
-  const cudaError_t e = launch_kernel(gemm_nvfp4_kernel<EPI>, dim3(2 * pairs), dim3(nv::kThreads), nv::kSmem, s, 2,
+  const cudaError_t e = launch_kernel(gemm_nvfp4_kernel<EPI>, dim3(2 * pairs), dim3(nv::kThreads), C::kSmem, s, 2,
                                       ma, mb, msfa, msfb, g);
   note_launch();
   return (e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess) ? 0 : -1;

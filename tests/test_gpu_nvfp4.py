@@ -247,3 +247,38 @@ def test_nvfp4_denoise_matches_oracle(kb):
     assert cosine(got, ref) >= 0.999, cosine(got, ref)
     assert rms(got - ref) / rms(ref) <= NV_REL, rms(got - ref) / rms(ref)
     assert max_err_ratio(got, ref) <= NV_MAX_ERR, max_err_ratio(got, ref)
+
+
+@pytest.mark.parametrize("batch,n_txt,grid,refs", [(1, 512, (64, 64), ()), (1, 512, (64, 64), ((64, 64),))])
+def test_nvfp4_block_full_size_sampled_rows(kb, nv_weights, batch, n_txt, grid, refs):
+    # the 1024x1024 text-to-image (4608 rows) and edit (8704 rows) joint
+    # blocks in NVFP4, in the launch configuration the bench times: each CTA
+    # pair of the persistent GEMMs walks dozens of tiles, so the scale warp's
+    # per-stage slots and barrier phases wrap many times. The oracle evaluates
+    # a sample of output rows, every row supplying keys and values.
+    wq, _, wd = nv_weights
+    n_img = grid[0] * grid[1]
+    n_ref = sum(h * ww for h, ww in refs)
+    n_total = n_txt + n_img + n_ref
+    seq = kb.make_seq(batch, n_txt, grid[0], grid[1], refs)
+    x = ki.tokens(1, f"nvblock.large.{n_total}", batch, n_total)
+    mod = ki.modulation_vectors(1, f"nvblock.large.{n_total}")
+    xd = to_f32(x)
+    pos = torch.empty((n_total, 4), dtype=torch.float32, device="cuda")
+    kb.klein_positions(seq, pos)
+    ws = workspace(kb.klein_block_workspace_size(batch, n_total))
+    kb.klein_block_forward(wd, xd, n_txt, n_img, pos, to_f32(mod), ws)
+    torch.cuda.synchronize()
+    got = host(xd)
+    rows = np.unique(np.concatenate([np.arange(0, n_total, 331), [0, n_txt - 1, n_txt, n_txt + n_img - 1,
+                                                                 n_total - 1]]))
+    rows = rows[rows < n_total]
+    ref = o.block(x, o.positions(n_txt, grid, refs), o.mode_of_rows(n_txt, n_img, n_ref),
+                  mod.astype(np.float64), wq, rows=rows)
+    g = got[:, rows]
+    d_got, d_ref = g - x[:, rows], ref - x[:, rows]
+    assert np.all(np.isfinite(g))
+    rel = rms(d_got - d_ref) / rms(d_ref)
+    assert rel <= NV_REL, rel
+    assert cosine(d_got, d_ref) >= 0.998
+    assert max_err_ratio(g, ref) <= NV_MAX_ERR, max_err_ratio(g, ref)
