@@ -88,6 +88,81 @@ def test_quantiser_bit_exact(kb, rows, cols, mode):
         assert not unpack_scales(full, pad, cols)[rows:].any()
 
 
+def _tie_rows(rows, cols, seed):
+    """Rows on which most codes are exact e2m1 ties. A row's maximum is
+    2688 * 2^j, so g = 2^j exactly; a block whose maximum is 6 s 2^j for an
+    e4m3 value s gets the block scale s and the step s 2^j exactly, and its
+    values t s 2^j (t a rounding boundary of e2m1: 0.25, 0.75, ... 5) are
+    exact ties of the round-to-nearest-even. Every other block holds the
+    bf16 neighbours (one bf16 step up or down) of boundaries and code
+    values."""
+    rng = np.random.default_rng(seed)
+    e4m3_s = np.array([2.0 ** -9, 0.015625, 0.125, 0.875, 1.0, 1.125, 1.5, 1.875, 3.0, 7.5, 13.0, 112.0, 240.0])
+    ties = np.array([6, .25, .75, 1.25, 1.75, 2.5, 3.5, 5, -.25, -.75, -1.25, -1.75, -2.5, -3.5, -5, -6])
+    near = np.array([6, .25, .75, 1.25, 1.75, 2.5, 3.5, 5, .5, 1, 1.5, 2, 3, 4, -.5, -4])
+    bump = np.array([0, 1, -1, 1, -1, 1, -1, 1, 1, -1, 1, -1, 1, -1, 1, -1], np.int64) << 16  # bf16 steps
+    a = np.empty((rows, cols), np.float32)
+    for r in range(rows):
+        j = int(rng.integers(-12, 6))
+        for blk in range(cols // 16):
+            s = 448.0 if blk == 0 else float(rng.choice(e4m3_s))
+            if blk % 2 == 0:
+                v = (ties * s * 2.0 ** j).astype(np.float32)
+            else:
+                v = (near * s * 2.0 ** j).astype(np.float32)
+                v = (v.view(np.uint32).astype(np.int64) + bump).astype(np.uint32).view(np.float32)
+            a[r, 16 * blk:16 * blk + 16] = rng.permutation(v)
+        a[r, 0] = 2688.0 * 2.0 ** j           # the row maximum: g = 2^j
+    assert np.array_equal(ki.round_to_bf16(a), a), "tie values must be bf16-representable"
+    return a
+
+
+@pytest.mark.parametrize("mode", ["rows", "matrix"])
+def test_quantiser_exact_ties(kb, mode):
+    # codes decided at exact ties and at bf16 neighbours of the e2m1 rounding
+    # boundaries: the same as the oracle's correctly rounded division
+    a = _tie_rows(64, 3072, 11)
+    if mode == "matrix":
+        a[1:, 0] = a[0, 0]                       # one maximum for the matrix: g = 2^j of row 0
+        a[1:] = np.minimum(np.abs(a[1:]), np.abs(a[0, 0])) * np.sign(a[1:])
+    m = kb.NVFP4_ROWS if mode == "rows" else kb.NVFP4_MATRIX
+    codes, sf, g = kb.klein_quantize_nvfp4(to_bf16(a), m)
+    torch.cuda.synchronize()
+    c_ref, s_ref, g_ref = nvfp4.quantize(a, per_row=(mode == "rows"))
+    np.testing.assert_array_equal(unpack_scales(sf.cpu().numpy(), 64, 3072), s_ref)
+    np.testing.assert_array_equal(unpack_codes(codes.cpu().numpy()), c_ref)
+    if mode == "rows":
+        # the construction did produce ties: values exactly halfway between
+        # two e2m1 codes, for a quarter of all values or more
+        step = fp8.e4m3_decode(s_ref) * np.asarray(g_ref, np.float64).reshape(-1, 1)
+        q = np.abs(a.reshape(64, -1, 16) / step[..., None])
+        assert np.isin(q, [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]).mean() >= 0.25
+
+
+def test_modln_nvfp4_exact_ties(kb):
+    # the fused modLN quantiser on rows whose modulated values are the tie
+    # rows above: x = 0 rows with shift = the tie row and scale = -1 give
+    # h = shift exactly, so every decision is the quantiser's
+    n_txt, n_img = 0, 64
+    ties = _tie_rows(1, ki.DIM, 12)[0]
+    x = np.zeros((1, n_img, ki.DIM), np.float32)
+    mod = np.zeros((3, 3, ki.DIM), np.float32)
+    mod[1, 0] = ties                               # image mode: shift
+    mod[1, 1] = -1.0                               # scale: (1 + scale) x^ = 0
+    codes = torch.empty((1, n_img, ki.DIM // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((1, 256 * ki.DIM // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty((1, n_img), dtype=torch.float32, device="cuda")
+    kb.klein_op_modln_nvfp4(to_f32(x), 0, n_img, n_txt, n_img, to_f32(mod), codes, sf, g)
+    torch.cuda.synchronize()
+    c_ref, s_ref, g_ref = nvfp4.quantize(ties[None, :].astype(np.float64), per_row=True)
+    got_c = unpack_codes(codes.cpu().numpy()[0])
+    got_s = unpack_scales(sf.cpu().numpy()[0], n_img, ki.DIM)
+    for r in range(n_img):
+        np.testing.assert_array_equal(got_c[r], c_ref[0])
+        np.testing.assert_array_equal(got_s[r], s_ref[0])
+    assert np.all(g.cpu().numpy() == np.float32(np.asarray(g_ref).ravel()[0]))
+
+
 def test_in_projection_order(kb):
     # a block's w_in in the NVFP4 in-projection order: q, k, v rows as they
     # are, then per 64-unit SwiGLU chunk its gate rows and its up rows
