@@ -141,3 +141,132 @@ def test_fp8_argument_errors_before_any_launch(kb):
     rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1 << 30, None)
     assert kb.STATUS[rc] == "KLEIN_ERR_INVALID_ARG"
     assert b"w_in_scale and w_out_scale" in kb.lib.klein_last_error()
+
+
+def _fake_model(kb, distilled=True):
+    """A model handle over aligned placeholder addresses: it passes
+    klein_model_create (which checks presence and alignment only) and serves
+    the argument checks below, each of which must fail before any launch
+    could read a weight."""
+    d = kb.KleinModelDesc()
+    d.n_stage1, d.n_joint = 0, 1
+    bw = kb.KleinBlockWeights(1 << 12, 2 << 12, 3 << 12, 4 << 12)
+    d.joint = ctypes.cast(ctypes.pointer(bw), ctypes.c_void_p)
+    d.img_in, d.t_mlp1, d.t_mlp2, d.final_mod, d.final_out = 5 << 12, 6 << 12, 7 << 12, 8 << 12, 9 << 12
+    if distilled:
+        d.tt_mlp1, d.tt_mlp2 = 10 << 12, 11 << 12
+    for st in range(2):
+        for m in range(2):
+            d.mod[st][m] = (12 + 2 * st + m) << 12
+    h = ctypes.c_void_p()
+    assert kb.lib.klein_model_create(ctypes.byref(h), ctypes.byref(d)) == 0
+    return h, bw          # the caller keeps bw alive: the model borrows it
+
+
+def test_denoise_and_stack_argument_errors(kb):
+    h, _bw = _fake_model(kb)
+    seq = kb.make_seq(1, 80, 8, 8)
+    seq2 = kb.make_seq(2, 80, 8, 8)
+    lat, txt, ws, big = 1 << 20, 2 << 20, 3 << 20, 1 << 40
+    den = kb.lib.klein_denoise
+
+    def st(rc):
+        return kb.STATUS[rc]
+
+    try:
+        assert st(den(None, lat, txt, None, 4, 1.0, 6.93, ctypes.byref(seq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_INVALID_ARG"
+        assert b"model is NULL" in kb.lib.klein_last_error()
+        assert st(den(h, lat, txt, None, 4, 1.0, 6.93, None, None, 0, ws, big, None)) == "KLEIN_ERR_INVALID_ARG"
+        bad = kb.make_seq(1, 80, 8, 8)
+        bad.batch = 0
+        assert st(den(h, lat, txt, None, 4, 1.0, 6.93, ctypes.byref(bad), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_SHAPE"
+        assert st(den(h, None, txt, None, 4, 1.0, 6.93, ctypes.byref(seq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_INVALID_ARG"
+        assert st(den(h, lat + 4, txt, None, 4, 1.0, 6.93, ctypes.byref(seq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_ALIGN"
+        # a reference in the sequence, but no reference weights in the model
+        rseq = kb.make_seq(1, 80, 8, 8, ((4, 4),))
+        assert st(den(h, lat, txt, 4 << 20, 4, 1.0, 6.93, ctypes.byref(rseq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_INVALID_ARG"
+        assert b"reference weights" in kb.lib.klein_last_error()
+        need = kb.lib.klein_stack_workspace_size(ctypes.byref(seq))
+        assert st(den(h, lat, txt, None, 4, 1.0, 6.93, ctypes.byref(seq), None, 0, ws, need - 1, None)) == \
+            "KLEIN_ERR_WORKSPACE"
+        for steps in (0, 1001):
+            assert st(den(h, lat, txt, None, steps, 1.0, 6.93, ctypes.byref(seq), None, 0, ws, big, None)) == \
+                "KLEIN_ERR_INVALID_ARG"
+        # guidance needs the (cond, uncond) pair as batch 2, and only then
+        assert st(den(h, lat, txt, None, 4, 3.5, 6.93, ctypes.byref(seq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_SHAPE"
+        assert st(den(h, lat, txt, None, 4, 1.0, 6.93, ctypes.byref(seq2), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_SHAPE"
+        assert st(den(h, lat, txt, None, 4, 1.0, 6.93, ctypes.byref(seq), lat + 8, 0, ws, big, None)) == \
+            "KLEIN_ERR_ALIGN"
+        assert st(den(h, lat, txt, None, 4, 1.0, 0.0, ctypes.byref(seq), None, 0, ws, big, None)) == \
+            "KLEIN_ERR_INVALID_ARG"
+        assert b"shift" in kb.lib.klein_last_error()
+        sf = kb.lib.klein_stack_forward
+        assert st(sf(h, lat, txt, None, ctypes.c_float(0.5), ctypes.c_float(0.4), ctypes.byref(seq), None, ws,
+                     big, None)) == "KLEIN_ERR_ALIGN"
+        assert st(sf(h, lat, txt, None, ctypes.c_float(0.5), ctypes.c_float(0.4), ctypes.byref(seq), 5 << 20, ws,
+                     need - 16, None)) == "KLEIN_ERR_WORKSPACE"
+    finally:
+        kb.lib.klein_model_destroy(h)
+
+
+def test_schedule_and_positions_argument_errors(kb):
+    out = (ctypes.c_float * 8)()
+    assert kb.STATUS[kb.lib.klein_sigma_schedule(0, 6.93, out)] == "KLEIN_ERR_INVALID_ARG"
+    assert kb.STATUS[kb.lib.klein_sigma_schedule(4, -1.0, out)] == "KLEIN_ERR_INVALID_ARG"
+    assert kb.STATUS[kb.lib.klein_sigma_schedule(4, 6.93, None)] == "KLEIN_ERR_INVALID_ARG"
+    seq = kb.make_seq(1, 80, 8, 8)
+    assert kb.STATUS[kb.lib.klein_positions(ctypes.byref(seq), None, None)] == "KLEIN_ERR_ALIGN"
+    assert kb.STATUS[kb.lib.klein_positions(ctypes.byref(seq), 4100, None)] == "KLEIN_ERR_ALIGN"
+    bad = kb.make_seq(1, 80, 8, 8, ((4, 4),))
+    bad.ref_w[0] = 0
+    assert kb.STATUS[kb.lib.klein_positions(ctypes.byref(bad), 4096, None)] == "KLEIN_ERR_SHAPE"
+    assert kb.lib.klein_stack_workspace_size(ctypes.byref(bad)) == 0
+
+
+def test_nvfp4_argument_errors_before_any_launch(kb):
+    q = kb.lib.klein_quantize_nvfp4
+    st = kb.STATUS
+    assert st[q(None, 4, 64, 0, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_INVALID_ARG"
+    assert st[q(4104, 4, 64, 0, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_ALIGN"
+    assert st[q(4096, 4, 64, 7, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_INVALID_ARG"      # mode
+    assert st[q(4096, 4, 48, 0, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_SHAPE"            # cols % 64
+    assert st[q(4096, 4, 12352, 0, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_SHAPE"         # cols > 12288
+    assert st[q(4096, 4, 3072, kb.NVFP4_IN_PROJ, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_SHAPE"
+    assert st[q(4096, 4, 64, 0, 4096 + 64, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_INVALID_ARG"    # codes overlap src
+    m = kb.lib.klein_op_modln_nvfp4
+    assert st[m(None, 1, 10, 0, 10, 5, 5, 4096, 9216, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_INVALID_ARG"
+    assert st[m(4096, 1, 10, 0, 10, 5, 5, 4096, 9214, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_ALIGN"
+    assert st[m(4096, 1, 10, 4, 10, 5, 5, 4096, 9216, 1 << 20, 2 << 20, 3 << 20, None)] == "KLEIN_ERR_SHAPE"
+    g = kb.lib.klein_op_gemm_nvfp4
+    ptrs = [(k + 1) << 20 for k in range(7)]
+    assert st[g(None, *ptrs[1:], 256, 256, 256, None)] == "KLEIN_ERR_INVALID_ARG"
+    assert st[g(*ptrs, 256, 200, 256, None)] == "KLEIN_ERR_SHAPE"     # N not a multiple of 128
+    assert st[g(*ptrs, 256, 256, 128, None)] == "KLEIN_ERR_SHAPE"     # K not a multiple of 256
+    # NVFP4 block weights need both block-scale arrays and both second-level scales
+    bw = kb.KleinBlockWeights(16, 32, 48, 64, None, None, 80, 96)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1 << 30, None)
+    assert st[rc] == "KLEIN_ERR_INVALID_ARG"
+    assert b"second-level scales" in kb.lib.klein_last_error()
+    bw = kb.KleinBlockWeights(16, 32, 48, 64, 112, 128, 80, None)
+    rc = kb.lib.klein_block_forward(ctypes.byref(bw), 256, 1, 10, 0, 10, 5, 5, 256, 256, 256, 1 << 30, None)
+    assert st[rc] == "KLEIN_ERR_INVALID_ARG"
+    assert b"w_in_sf and w_out_sf" in kb.lib.klein_last_error()
+
+
+def test_attention_argument_errors_before_any_launch(kb):
+    a = kb.lib.klein_op_attention
+    st = kb.STATUS
+    p = [(k + 1) << 20 for k in range(4)]
+    assert st[a(None, p[1], p[2], 1, 128, 128, p[3], 3072, None)] == "KLEIN_ERR_INVALID_ARG"
+    assert st[a(*p[:3], 1, 128, 128, p[3], 3076, None)] == "KLEIN_ERR_ALIGN"          # out_ld % 8
+    assert st[a(*p[:3], 1, 128, 120, p[3], 3072, None)] == "KLEIN_ERR_SHAPE"          # rows_pad < rows
+    assert st[a(*p[:3], 1, 128, 132, p[3], 3072, None)] == "KLEIN_ERR_SHAPE"          # rows_pad % 8
+    assert st[a(*p[:3], 1, 128, 128, p[3], 2048, None)] == "KLEIN_ERR_SHAPE"          # out_ld < 3072
+    assert st[a(*p[:3], 0, 128, 128, p[3], 3072, None)] == "KLEIN_ERR_SHAPE"
