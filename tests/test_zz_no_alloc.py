@@ -125,3 +125,26 @@ def test_static_scratch_fp8_block_at_the_size_limit(kb):
         torch.cuda.synchronize()
         np.testing.assert_array_equal(host(got), host(ref))
     assert kb.klein_device_status()[0] == 0
+
+
+def test_static_scratch_nvfp4_block_at_the_size_limit(kb):
+    # NVFP4 weights, batch 2 x 128 rows = the array's limit of 256 rows; the
+    # block scales of both GEMM inputs are laid out per batch item over 256
+    # rows (the GEMM's row tile), which the fixed array reserves as well, so
+    # the result is the workspace path's, bit for bit
+    w = kb.quantize_block_nvfp4(upload_block(ki.block_weights(0, "joint.0")))
+    n_txt, gh, gw = 64, 8, 8
+    n = n_txt + gh * gw                   # 128 rows
+    x = ki.tokens(1, "no_alloc.nvfp4", 2, n)
+    mod = to_f32(ki.modulation_vectors(1, "no_alloc.nvfp4"))
+    pos = torch.empty((n, 4), dtype=torch.float32, device="cuda")
+    kb.klein_positions(kb.make_seq(2, n_txt, gh, gw), pos)
+    ref = to_f32(x)
+    ws = workspace(kb.klein_block_workspace_size(2, n))
+    kb.klein_block_forward(w, ref, n_txt, gh * gw, pos, mod, ws)
+    for _ in range(2):
+        got = to_f32(x)
+        kb.klein_block_forward_static(w, got, n_txt, gh * gw, pos, mod)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(got), host(ref))
+    assert kb.klein_device_status()[0] == 0
