@@ -56,13 +56,13 @@ FP8_OVER_BF16 = 2.0
 FP4_OVER_BF16 = 4.0
 PEAK_RATIO = {"bf16": 1.0, "fp8": FP8_OVER_BF16, "nvfp4": FP4_OVER_BF16}
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one bf16 in-projection GEMM
-# launch (gemm_pair_kernel<2, 0>) over 512 + 4096 rows, the launch shape of
-# every joint block of the 1024x1024 denoise, from an ncu capture of
-# `bench.py --workload block` (one joint block; its summary is kept with the
-# other kernel profiles). Must be re-captured (or set to None) whenever that
-# kernel changes.
-GEMM_IN_TRAFFIC_BYTES = 357.31e6
+# dram__bytes_read.sum + dram__bytes_write.sum of one in-projection GEMM
+# launch over 512 + 4096 rows, the launch shape of every joint block of the
+# 1024x1024 denoise, per block precision, from ncu captures of
+# `bench.py --workload block [--precision ...]` (one joint block; the summary
+# is kept with the other kernel profiles). Must be re-captured (or set to
+# None) whenever that kernel changes.
+GEMM_IN_TRAFFIC_BYTES = {"bf16": 357.31e6, "fp8": 233.06e6, "nvfp4": 175.53e6}
 
 
 def load_peaks():
@@ -591,7 +591,7 @@ def run_ours(args):
                           f"{', ' + args.precision if fp8 else ''}; {gi_rows} rows x 3072 -> 27648 per launch)",
                 "bound": "tensor", "achieved": achieved, "peak": gi_peak, "unit": "TFLOP/s",
                 "frac": achieved / gi_peak,
-                "traffic": GEMM_IN_TRAFFIC_BYTES if (gi_rows == 4608 and not fp8) else None,
+                "traffic": GEMM_IN_TRAFFIC_BYTES.get(args.precision) if gi_rows == 4608 else None,
                 "traffic_unit": "bytes per launch (ncu dram read + write of the same 4608-row launch)",
                 "algorithmic_flop_per_launch": gi_rows * 2.0 * DIM * (3 * DIM + 2 * MLP),
                 "avg_launch_ms": gi_avg_ms, "launches": gi_n,
