@@ -84,7 +84,9 @@ int launch_gemm(int bn, int epi, const CUtensorMap& map_a, const CUtensorMap& ma
 // [batch][rows][K/2] with scale atoms over round_up(rows, 256) rows per batch
 // item, B codes [n_rows_b][K/2] with scale atoms (n_rows_b a multiple of
 // 128); epi is kEpiF32, kEpiQKV (tile n < 72: head n % 24 of q, k, v; else
-// 64 SwiGLU hidden units, B rows 64 gate then 64 up) or kEpiResid.
+// 64 SwiGLU hidden units, B rows 64 gate then 64 up) or kEpiResid (256 x 256
+// tiles: n_tiles must be even). Returns 0, -1 (launch), -2 (tensor map) or
+// -3 (shape).
 int launch_gemm_nvfp4(int epi, const void* a, long long a_ld, const void* a_sf, const void* b, const void* b_sf,
                       const GemmArgs& args, int n_rows_b, cudaStream_t stream);
 // NVFP4 quantisation of `batch` bf16 matrices [rows][cols] (see nvfp4.cu);

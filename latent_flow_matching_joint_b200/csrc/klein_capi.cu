@@ -272,6 +272,7 @@ static int block_impl_nvfp4(const klein_block_weights* wt, float* x, int batch, 
   // the codes sit at the start of each bf16 [attention | SwiGLU] row (pitch 24576 bytes)
   rc = launch_gemm_nvfp4(kEpiResid, w.a_out, (long long)kOutK * 2, w.sf_o, wt->w_out, wt->w_out_sf, o, kDim, s);
   if (rc == -2) return fail(KLEIN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  if (rc == -3) return fail(KLEIN_ERR_SHAPE, "the out-projection's N must be a multiple of 256");
   if (rc) return cuda_fail("out-projection GEMM launch");
   prof_end(pi, s);
   return KLEIN_OK;

@@ -744,7 +744,7 @@ template <int EPI>
 static int launch_nvfp4_one(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msfa,
                             const CUtensorMap& msfb, const GemmArgs& g, cudaStream_t s) {
   using C = nv::Cfg<EPI == kEpiResid>;
-  if (g.n_tiles % C::kHalves != 0) return -2;  // a wide tile covers two 128-column tiles
+  if (g.n_tiles % C::kHalves != 0) return -3;  // a wide tile covers two 128-column tiles
   static int max_pairs_dev[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0) return -1;
